@@ -1,0 +1,474 @@
+// libtq C ABI: argument validation and kernel dispatch.  This is the single
+// CUDA translation unit of the library (the kernels live in the included
+// headers), so the device error word has one definition.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "tq_attention.cuh"
+#include "tq_device.cuh"
+#include "tq_encode.cuh"
+#include "tq_gemm.cuh"
+#include "tq_internal.h"
+#include "tq_scores.cuh"
+
+namespace tq {
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline size_t dtype_size(int dt) { return dt == TQ_F32 ? 4 : 2; }
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <typename T, bool PROD>
+cudaError_t encode_hadamard_dispatch(const QParams& qp, const T* x, int64_t ld, int64_t seg_len,
+                                     int64_t seg_cap, int64_t n_seg, int layout, uint32_t* codes,
+                                     uint32_t* signs, float* norms, float* rnorms,
+                                     cudaStream_t st) {
+  const int64_t bps = ceil_div(seg_len, 32);
+  const int64_t tasks = n_seg * bps;
+  if (tasks == 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>(ceil_div(tasks, 4), (int64_t)num_sms() * 16);
+  const int A = qp.d_pad / 32;
+#define TQ_ENC(AA)                                                                          \
+  case AA:                                                                                  \
+    encode_hadamard_kernel<AA, T, PROD><<<(unsigned)blocks, 128, 0, st>>>(                  \
+        qp, x, ld, seg_len, seg_cap, bps, tasks, layout, codes, signs, norms, rnorms);      \
+    break;
+  switch (A) {
+    TQ_ENC(1)
+    TQ_ENC(2)
+    TQ_ENC(4)
+    TQ_ENC(8)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef TQ_ENC
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t encode_dense(const QParams& qp, bool prod, const T* x, int64_t ld, int64_t n_vec,
+                         int64_t seg_len, int64_t seg_cap, int layout, uint32_t* codes,
+                         uint32_t* signs, float* norms, float* rnorms, float* ws, int64_t chunk,
+                         cudaStream_t st) {
+  const int d = qp.d;
+  float* xh = ws;                          // [chunk][d]
+  float* y = ws + (size_t)chunk * d;       // [chunk][d]  (y, then r)
+  float* z = y + (size_t)chunk * d;        // [chunk][m]
+  int64_t row = 0;
+  while (row < n_vec) {
+    // a chunk never crosses a segment boundary and starts on a 32-block
+    const int64_t s = row / seg_len, t = row % seg_len;
+    const int64_t rows = std::min<int64_t>(chunk, seg_len - t);
+    normalize_rows_kernel<T><<<(unsigned)ceil_div(rows, 4), 128, 0, st>>>(
+        x, ld, d, seg_len, seg_cap, row, rows, xh, norms);
+    cudaError_t e = gemm_abt_f32(xh, qp.Pi, y, (int)rows, d, d, st);
+    if (e != cudaSuccess) return e;
+    quantize_rows_kernel<<<(unsigned)ceil_div(ceil_div(rows, 32), 4), 128, 0, st>>>(
+        qp, y, seg_len, seg_cap, row, rows, layout, prod, codes, rnorms);
+    if (prod) {
+      e = gemm_abt_f32(y, qp.S, z, (int)rows, qp.m, d, st);
+      if (e != cudaSuccess) return e;
+      pack_signs_kernel<<<(unsigned)ceil_div(rows, 4), 128, 0, st>>>(z, qp.m, seg_len, seg_cap,
+                                                                     row, rows, signs);
+    }
+    (void)s;
+    row += rows;
+  }
+  return cudaGetLastError();
+}
+
+constexpr int64_t kDenseChunk = 32768;
+
+size_t encode_workspace_bytes(const QParams& qp, bool prod, int64_t n_vec) {
+  if (qp.rot != TQ_ROT_DENSE || n_vec == 0) return 0;
+  const int64_t chunk = std::min<int64_t>(kDenseChunk, round_up(n_vec, 32));
+  return round_up((size_t)chunk * (2 * qp.d + (prod ? qp.m : 0)) * sizeof(float), 256);
+}
+
+}  // namespace
+
+int launch_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_vec, int64_t ld,
+                  int64_t seg_len, int64_t seg_cap, int layout, uint32_t* codes, uint32_t* signs,
+                  float* norms, float* rnorms, void* ws, void* stream) {
+  const int64_t n_seg = n_vec / seg_len;
+  cudaStream_t st = S(stream);
+  if (qp.rot == TQ_ROT_DENSE) {
+    const int64_t chunk = std::min<int64_t>(kDenseChunk, round_up(n_vec, 32));
+    float* w = (float*)ws;
+    switch (dt) {
+      case TQ_F32: return encode_dense(qp, prod, (const float*)x, ld, n_vec, seg_len, seg_cap, layout, codes, signs, norms, rnorms, w, chunk, st);
+      case TQ_F16: return encode_dense(qp, prod, (const __half*)x, ld, n_vec, seg_len, seg_cap, layout, codes, signs, norms, rnorms, w, chunk, st);
+      default: return encode_dense(qp, prod, (const __nv_bfloat16*)x, ld, n_vec, seg_len, seg_cap, layout, codes, signs, norms, rnorms, w, chunk, st);
+    }
+  }
+#define TQ_DT(T)                                                                                  \
+  return prod ? encode_hadamard_dispatch<T, true>(qp, (const T*)x, ld, seg_len, seg_cap, n_seg,   \
+                                                  layout, codes, signs, norms, rnorms, st)        \
+              : encode_hadamard_dispatch<T, false>(qp, (const T*)x, ld, seg_len, seg_cap, n_seg,  \
+                                                   layout, codes, signs, norms, rnorms, st);
+  switch (dt) {
+    case TQ_F32: TQ_DT(float)
+    case TQ_F16: TQ_DT(__half)
+    default: TQ_DT(__nv_bfloat16)
+  }
+#undef TQ_DT
+}
+
+int launch_decode(const QParams& qp, int layout, const uint32_t* codes, const uint32_t* signs,
+                  const float* norms, const float* rnorms, int64_t n_vec, int64_t seg_len,
+                  int64_t seg_cap, float* out, int64_t ldo, void* stream) {
+  cudaStream_t st = S(stream);
+  const unsigned blocks = (unsigned)ceil_div(n_vec, 4);
+  if (qp.rot == TQ_ROT_DENSE) {
+    decode_dense_kernel<<<blocks, 128, 4 * qp.d * sizeof(float), st>>>(
+        qp, layout, codes, signs, norms, rnorms, n_vec, seg_len, seg_cap, out, ldo);
+    return cudaGetLastError();
+  }
+  switch (qp.d_pad / 32) {
+#define TQ_DEC(AA)                                                                             \
+  case AA:                                                                                     \
+    decode_hadamard_kernel<AA><<<blocks, 128, 0, st>>>(qp, layout, codes, signs, norms, rnorms, \
+                                                       n_vec, seg_len, seg_cap, out, ldo);     \
+    break;
+    TQ_DEC(1)
+    TQ_DEC(2)
+    TQ_DEC(4)
+    TQ_DEC(8)
+#undef TQ_DEC
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+int launch_query_prep(const QParams& qp, const float* q, int64_t nq, int64_t ldq, float* qrot,
+                      float* u, void* stream) {
+  cudaStream_t st = S(stream);
+  const unsigned blocks = (unsigned)ceil_div(nq, 4);
+  if (nq == 0) return cudaSuccess;
+  if (qp.rot == TQ_ROT_DENSE) {
+    query_prep_dense_kernel<<<blocks, 128, 4 * 2 * qp.d * sizeof(float), st>>>(qp, q, nq, ldq,
+                                                                               qrot, u);
+    return cudaGetLastError();
+  }
+  switch (qp.d_pad / 32) {
+#define TQ_QP(AA)                                                                                \
+  case AA:                                                                                       \
+    query_prep_hadamard_kernel<AA><<<blocks, 128, 0, st>>>(qp, q, nq, ldq, qrot, u);             \
+    break;
+    TQ_QP(1)
+    TQ_QP(2)
+    TQ_QP(4)
+    TQ_QP(8)
+#undef TQ_QP
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+namespace {
+int score_query_tile(const QParams& qp) {
+  const size_t per_q = (size_t)(qp.d_pad + qp.m) * sizeof(float);
+  int qt = (int)std::min<size_t>(32, (96 * 1024) / per_q);
+  return std::max(qt, 1);
+}
+}  // namespace
+
+int launch_scores(const QParams& qp, const float* qrot, const float* u, int64_t nq,
+                  const uint32_t* codes, const uint32_t* signs, const float* norms,
+                  const float* rnorms, int64_t n_vec, float* scores, void* stream) {
+  if (nq == 0 || n_vec == 0) return cudaSuccess;
+  const int qt = score_query_tile(qp);
+  const size_t smem = (size_t)qt * (qp.d_pad + qp.m) * sizeof(float);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
+    attr_set = true;
+  }
+  dim3 grid((unsigned)ceil_div(n_vec, kScoreThreads), (unsigned)ceil_div(nq, qt));
+  scores_kernel<<<grid, kScoreThreads, smem, S(stream)>>>(qp, qrot, u, nq, qt, codes, signs, norms,
+                                                          rnorms, n_vec, scores);
+  return cudaGetLastError();
+}
+
+int launch_topk(const float* scores, int64_t nq, int64_t n_vec, int topk, float* top_s,
+                int64_t* top_i, void* stream) {
+  if (nq == 0) return cudaSuccess;
+  topk_kernel<<<(unsigned)nq, kTopkThreads, 0, S(stream)>>>(scores, n_vec, topk, top_s, top_i);
+  return cudaGetLastError();
+}
+
+size_t attention_workspace(const QParams& kp, const QParams& vp, int L, int B, int Hq, int Hkv,
+                           int64_t seq, int* chunk_out, int* n_chunks_out) {
+  const int64_t groups = (int64_t)L * B * Hkv;
+  const int G = Hq / Hkv;
+  const int64_t target = (int64_t)num_sms() * 32;
+  int64_t n_chunks = std::max<int64_t>(1, ceil_div(target, std::max<int64_t>(groups, 1)));
+  int64_t chunk = round_up(ceil_div(seq, n_chunks), 32);
+  chunk = std::max<int64_t>(chunk, 256);
+  n_chunks = ceil_div(seq, chunk);
+  if (chunk_out) *chunk_out = (int)chunk;
+  if (n_chunks_out) *n_chunks_out = (int)n_chunks;
+  const int64_t nq = (int64_t)L * B * Hq;
+  size_t bytes = round_up((size_t)nq * kp.d_pad * 4, 256) + round_up((size_t)nq * kp.m * 4, 256) +
+                 round_up((size_t)groups * n_chunks * G * (vp.d_pad + 2) * 4, 256);
+  return bytes;
+}
+
+int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q, int L, int B,
+                            int Hq, int Hkv, int64_t seq, int64_t cap, float scale,
+                            const uint32_t* kcodes, const uint32_t* ksigns, const float* knorms,
+                            const float* krnorms, const uint32_t* vcodes, const float* vnorms,
+                            float* out, void* ws, void* stream) {
+  cudaStream_t st = S(stream);
+  int chunk = 0, n_chunks = 0;
+  attention_workspace(kp, vp, L, B, Hq, Hkv, seq, &chunk, &n_chunks);
+  const int64_t nq = (int64_t)L * B * Hq;
+  char* w = (char*)ws;
+  float* qrot = (float*)w;
+  w += round_up((size_t)nq * kp.d_pad * 4, 256);
+  float* u = (float*)w;
+  w += round_up((size_t)nq * kp.m * 4, 256);
+  float* part = (float*)w;
+  int e = launch_query_prep(kp, q, nq, kp.d, qrot, u, stream);
+  if (e != cudaSuccess) return e;
+  AttnShape sh;
+  sh.G = Hq / Hkv;
+  sh.groups = L * B * Hkv;
+  sh.n_chunks = n_chunks;
+  sh.chunk = chunk;
+  sh.seq = seq;
+  sh.cap = cap;
+  sh.scale = scale;
+  const size_t smem = (size_t)sh.G * (kp.d_pad + kp.m) * sizeof(float);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(attention_chunk_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+    cudaFuncSetAttribute(attention_chunk_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+    attr_set = true;
+  }
+  dim3 grid((unsigned)n_chunks, (unsigned)sh.groups);
+  if (kp.d_pad <= 128)
+    attention_chunk_kernel<1><<<grid, kAttnThreads, smem, st>>>(kp, vp, sh, qrot, u, kcodes, ksigns, knorms, krnorms, vcodes, vnorms, part);
+  else
+    attention_chunk_kernel<2><<<grid, kAttnThreads, smem, st>>>(kp, vp, sh, qrot, u, kcodes, ksigns, knorms, krnorms, vcodes, vnorms, part);
+  cudaError_t ce = cudaGetLastError();
+  if (ce != cudaSuccess) return ce;
+  const unsigned cblocks = (unsigned)ceil_div((int64_t)sh.groups * sh.G, 4);
+  switch (vp.d_pad / 32) {
+#define TQ_CMB(AA)                                                                                 \
+  case AA:                                                                                         \
+    attention_combine_hadamard_kernel<AA><<<cblocks, 128, 0, st>>>(vp, sh, part, out, Hq, Hkv);    \
+    break;
+    TQ_CMB(1)
+    TQ_CMB(2)
+    TQ_CMB(4)
+    TQ_CMB(8)
+#undef TQ_CMB
+    default:
+      return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+int read_and_clear_device_error(void* stream, unsigned* err) {
+  cudaError_t e = cudaStreamSynchronize(S(stream));
+  if (e != cudaSuccess) return e;
+  unsigned v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e != cudaSuccess) return e;
+  const unsigned zero = 0;
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  *err = v;
+  return e;
+}
+
+}  // namespace tq
+
+// ====================================================================== C ABI
+
+namespace {
+
+tq_status cuda_status(int e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
+
+tq_status check_segments(int64_t n_vec, int64_t* seg_len, int64_t* seg_cap, bool block) {
+  if (n_vec < 0) return TQ_ERR_INVALID_ARG;
+  if (*seg_len == 0) *seg_len = n_vec;
+  if (*seg_len < 0) return TQ_ERR_INVALID_ARG;
+  if (n_vec == 0) return TQ_OK;
+  if (n_vec % *seg_len != 0) return TQ_ERR_INVALID_ARG;
+  if (*seg_cap == 0) *seg_cap = block ? (*seg_len + 31) / 32 * 32 : *seg_len;
+  if (*seg_cap < *seg_len) return TQ_ERR_INVALID_ARG;
+  if (block && *seg_cap % 32 != 0) return TQ_ERR_INVALID_ARG;
+  return TQ_OK;
+}
+
+tq_status check_encode_common(const tq_params* p, const void* x, tq_dtype dt, int64_t n_vec,
+                              int64_t ld, int64_t* seg_len, int64_t* seg_cap, int layout) {
+  if (!p) return TQ_ERR_INVALID_ARG;
+  if (dt != TQ_F32 && dt != TQ_F16 && dt != TQ_BF16) return TQ_ERR_INVALID_ARG;
+  if (layout != TQ_LAYOUT_ROW && layout != TQ_LAYOUT_BLOCK32) return TQ_ERR_INVALID_ARG;
+  tq_status s = check_segments(n_vec, seg_len, seg_cap, layout == TQ_LAYOUT_BLOCK32);
+  if (s != TQ_OK) return s;
+  if (n_vec == 0) return TQ_OK;
+  if (!x || ld < p->q.d) return TQ_ERR_INVALID_ARG;
+  if (!tq::aligned16(x) || (ld * (int64_t)tq::dtype_size(dt)) % 16 != 0) return TQ_ERR_INVALID_ARG;
+  if (p->q.rot == TQ_ROT_DENSE && layout == TQ_LAYOUT_BLOCK32 && *seg_len % 32 != 0)
+    return TQ_ERR_UNSUPPORTED;
+  return TQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tq_status tq_encode_workspace_size(const tq_params* p, int64_t n_vec, size_t* bytes) {
+  if (!p || !bytes || n_vec < 0) return TQ_ERR_INVALID_ARG;
+  *bytes = tq::encode_workspace_bytes(p->q, p->mode == TQ_MODE_PROD, n_vec);
+  return TQ_OK;
+}
+
+tq_status tq_encode_mse(const tq_params* p, const void* x, tq_dtype dt, int64_t n_vec, int64_t ld,
+                        int64_t seg_len, int64_t seg_cap, tq_layout layout, uint32_t* codes,
+                        float* norms, void* ws, size_t ws_bytes, void* stream) {
+  tq_status s = check_encode_common(p, x, dt, n_vec, ld, &seg_len, &seg_cap, layout);
+  if (s != TQ_OK) return s;
+  if (p->mode != TQ_MODE_MSE) return TQ_ERR_INVALID_ARG;
+  if (n_vec == 0) return TQ_OK;
+  if (!codes || !norms || !tq::aligned16(codes) || !tq::aligned16(norms)) return TQ_ERR_INVALID_ARG;
+  const size_t need = tq::encode_workspace_bytes(p->q, false, n_vec);
+  if (need > 0 && (!ws || ws_bytes < need || !tq::aligned256(ws))) return TQ_ERR_WORKSPACE;
+  return cuda_status(tq::launch_encode(p->q, false, x, dt, n_vec, ld, seg_len, seg_cap, layout,
+                                       codes, nullptr, norms, nullptr, ws, stream));
+}
+
+tq_status tq_encode_prod(const tq_params* p, const void* x, tq_dtype dt, int64_t n_vec, int64_t ld,
+                         int64_t seg_len, int64_t seg_cap, uint32_t* codes, uint32_t* signs,
+                         float* norms, float* rnorms, void* ws, size_t ws_bytes, void* stream) {
+  tq_status s = check_encode_common(p, x, dt, n_vec, ld, &seg_len, &seg_cap, TQ_LAYOUT_ROW);
+  if (s != TQ_OK) return s;
+  if (p->mode != TQ_MODE_PROD) return TQ_ERR_INVALID_ARG;
+  if (n_vec == 0) return TQ_OK;
+  if (!codes || !signs || !norms || !rnorms) return TQ_ERR_INVALID_ARG;
+  if (!tq::aligned16(codes) || !tq::aligned16(signs) || !tq::aligned16(norms) || !tq::aligned16(rnorms))
+    return TQ_ERR_INVALID_ARG;
+  const size_t need = tq::encode_workspace_bytes(p->q, true, n_vec);
+  if (need > 0 && (!ws || ws_bytes < need || !tq::aligned256(ws))) return TQ_ERR_WORKSPACE;
+  return cuda_status(tq::launch_encode(p->q, true, x, dt, n_vec, ld, seg_len, seg_cap,
+                                       TQ_LAYOUT_ROW, codes, signs, norms, rnorms, ws, stream));
+}
+
+tq_status tq_decode(const tq_params* p, tq_layout layout, const uint32_t* codes,
+                    const uint32_t* signs, const float* norms, const float* rnorms, int64_t n_vec,
+                    int64_t seg_len, int64_t seg_cap, float* out, int64_t ldo, void* stream) {
+  if (!p) return TQ_ERR_INVALID_ARG;
+  if (layout != TQ_LAYOUT_ROW && layout != TQ_LAYOUT_BLOCK32) return TQ_ERR_INVALID_ARG;
+  tq_status s = check_segments(n_vec, &seg_len, &seg_cap, layout == TQ_LAYOUT_BLOCK32);
+  if (s != TQ_OK) return s;
+  if (n_vec == 0) return TQ_OK;
+  if (!codes || !norms || !out || ldo < p->q.d) return TQ_ERR_INVALID_ARG;
+  if (signs && (p->mode != TQ_MODE_PROD || !rnorms)) return TQ_ERR_INVALID_ARG;
+  if (!tq::aligned16(codes) || !tq::aligned16(norms) || !tq::aligned16(out)) return TQ_ERR_INVALID_ARG;
+  return cuda_status(tq::launch_decode(p->q, layout, codes, signs, norms, rnorms, n_vec, seg_len,
+                                       seg_cap, out, ldo, stream));
+}
+
+tq_status tq_scores_workspace_size(const tq_params* kp, int64_t nq, int64_t n_vec, int topk,
+                                   size_t* bytes) {
+  if (!kp || !bytes || nq < 0 || n_vec < 0 || topk < 0) return TQ_ERR_INVALID_ARG;
+  size_t b = tq::round_up((size_t)nq * kp->q.d_pad * 4, 256) + tq::round_up((size_t)nq * kp->q.m * 4, 256);
+  if (topk > 0) b += tq::round_up((size_t)nq * n_vec * 4, 256);
+  *bytes = b;
+  return TQ_OK;
+}
+
+tq_status tq_scores(const tq_params* kp, const float* q, int64_t nq, int64_t ldq,
+                    const uint32_t* codes, const uint32_t* signs, const float* norms,
+                    const float* rnorms, int64_t n_vec, float* scores, int topk, float* top_s,
+                    int64_t* top_i, void* ws, size_t ws_bytes, void* stream) {
+  if (!kp || kp->mode != TQ_MODE_PROD) return TQ_ERR_INVALID_ARG;
+  if (nq < 0 || n_vec < 0 || topk < 0 || topk > tq::kTopkMax) return TQ_ERR_INVALID_ARG;
+  if (!scores && topk == 0) return TQ_ERR_INVALID_ARG;
+  if (topk > 0 && (!top_s || !top_i || topk > n_vec)) return TQ_ERR_INVALID_ARG;
+  if (nq == 0 || n_vec == 0) return TQ_OK;
+  if (!q || ldq < kp->q.d || !codes || !signs || !norms || !rnorms) return TQ_ERR_INVALID_ARG;
+  size_t need = 0;
+  tq_scores_workspace_size(kp, nq, n_vec, topk, &need);
+  if (!ws || ws_bytes < need || !tq::aligned256(ws)) return TQ_ERR_WORKSPACE;
+  char* w = (char*)ws;
+  float* qrot = (float*)w;
+  w += tq::round_up((size_t)nq * kp->q.d_pad * 4, 256);
+  float* u = (float*)w;
+  w += tq::round_up((size_t)nq * kp->q.m * 4, 256);
+  float* full = topk > 0 ? (float*)w : scores;
+  int e = tq::launch_query_prep(kp->q, q, nq, ldq, qrot, u, stream);
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
+  e = tq::launch_scores(kp->q, qrot, u, nq, codes, signs, norms, rnorms, n_vec, full, stream);
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
+  if (topk > 0) {
+    if (scores && scores != full) {
+      e = cudaMemcpyAsync(scores, full, (size_t)nq * n_vec * 4, cudaMemcpyDeviceToDevice,
+                          tq::S(stream));
+      if (e != cudaSuccess) return TQ_ERR_CUDA;
+    }
+    e = tq::launch_topk(full, nq, n_vec, topk, top_s, top_i, stream);
+    if (e != cudaSuccess) return TQ_ERR_CUDA;
+  }
+  return TQ_OK;
+}
+
+tq_status tq_decode_attention_workspace_size(const tq_params* kp, const tq_params* vp, int L,
+                                             int B, int Hq, int Hkv, int64_t seq,
+                                             size_t* bytes) {
+  if (!kp || !vp || !bytes || L < 1 || B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0 || seq < 1)
+    return TQ_ERR_INVALID_ARG;
+  *bytes = tq::attention_workspace(kp->q, vp->q, L, B, Hq, Hkv, seq, nullptr, nullptr);
+  return TQ_OK;
+}
+
+tq_status tq_decode_attention(const tq_params* kp, const tq_params* vp, const float* q, int L,
+                              int B, int Hq, int Hkv, int64_t seq, int64_t cap, float scale,
+                              const uint32_t* kcodes, const uint32_t* ksigns, const float* knorms,
+                              const float* krnorms, const uint32_t* vcodes, const float* vnorms,
+                              float* out, void* ws, size_t ws_bytes, void* stream) {
+  if (!kp || !vp || kp->mode != TQ_MODE_PROD || vp->mode != TQ_MODE_MSE) return TQ_ERR_INVALID_ARG;
+  if (kp->q.d != vp->q.d || kp->q.rot != vp->q.rot) return TQ_ERR_INVALID_ARG;
+  if (kp->q.rot != TQ_ROT_HADAMARD) return TQ_ERR_UNSUPPORTED;
+  if (L < 1 || B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0) return TQ_ERR_INVALID_ARG;
+  if (Hq / Hkv > tq::kAttnMaxG) return TQ_ERR_UNSUPPORTED;
+  if (seq < 1 || cap < seq || cap % 32 != 0) return TQ_ERR_INVALID_ARG;
+  if (!q || !kcodes || !ksigns || !knorms || !krnorms || !vcodes || !vnorms || !out)
+    return TQ_ERR_INVALID_ARG;
+  if (!tq::aligned16(q) || !tq::aligned16(kcodes) || !tq::aligned16(vcodes) || !tq::aligned16(out))
+    return TQ_ERR_INVALID_ARG;
+  size_t need = tq::attention_workspace(kp->q, vp->q, L, B, Hq, Hkv, seq, nullptr, nullptr);
+  if (!ws || ws_bytes < need || !tq::aligned256(ws)) return TQ_ERR_WORKSPACE;
+  return cuda_status(tq::launch_decode_attention(kp->q, vp->q, q, L, B, Hq, Hkv, seq, cap, scale,
+                                                 kcodes, ksigns, knorms, krnorms, vcodes, vnorms,
+                                                 out, ws, stream));
+}
+
+tq_status tq_sync_check(void* stream) {
+  unsigned err = 0;
+  if (tq::read_and_clear_device_error(stream, &err) != cudaSuccess) return TQ_ERR_CUDA;
+  if (err == 0) return TQ_OK;
+  return err == TQ_ERR_TIMEOUT ? TQ_ERR_TIMEOUT : TQ_ERR_INTERNAL;
+}
+
+}  // extern "C"

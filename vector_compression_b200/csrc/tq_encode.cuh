@@ -1,0 +1,270 @@
+// Encode kernels: TurboQuant-MSE and TurboQuant-prod.
+//
+// Per vector (TurboQuant blog notes, Q_MSE and the definition of Q_prod;
+// explainer §6 and §8):
+//   n = ||x||, y = Pi (x / n), idx_j = #{k : B_k < y_j}, codes = pack(idx);
+//   Q_prod additionally: r = y - C[idx], rho = ||r||, sign bits of S r.
+//
+// Hadamard rotation (explainer §0.9, DRIVE's randomized Hadamard; FastVQ's
+// sign-flipped Hadamard with padding): one warp per vector, lane l holding
+// coordinates 32a + l; the transform runs in registers and shuffles.
+// Dense rotation: the rotation and the QJL projection run as GEMMs over a
+// chunk of vectors (tq_gemm.cuh), with the per-vector steps here.
+#pragma once
+
+#include "tq_device.cuh"
+
+namespace tq {
+
+// Shared per-CTA copy of the codebook (dynamic indexing by lane).
+struct SmemCodebook {
+  float c[kMaxLevels];
+  float b[kMaxLevels];
+};
+
+__device__ __forceinline__ void load_codebook(SmemCodebook& cb, const QParams& qp) {
+  if (threadIdx.x < kMaxLevels) {
+    cb.c[threadIdx.x] = qp.centroids[threadIdx.x];
+    cb.b[threadIdx.x] = qp.boundaries[threadIdx.x];
+  }
+}
+
+// Quantize the rotated unit vector held by the warp (lane l: coordinates
+// 32a + l in y[a]) and emit ROW code words (lane w < k*A ends with word w in
+// *row_word) or accumulate BLOCK32 bits for vector slot t.  Returns idx in
+// idx[a].  Coordinates >= d_pad are not present (d_pad = 32 A).
+template <int A>
+__device__ __forceinline__ void quantize_pack(const float (&y)[A], int (&idx)[A],
+                                              const SmemCodebook& cb, int k, int lane,
+                                              uint32_t* row_word, uint32_t (*blk)[A], int t,
+                                              bool block_layout) {
+  const int nb = (1 << k) - 1;
+#pragma unroll
+  for (int a = 0; a < A; ++a) idx[a] = quantize_index(y[a], cb.b, nb);
+  if (block_layout) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      if (p < k) {
+#pragma unroll
+        for (int a = 0; a < A; ++a) blk[p][a] |= (uint32_t)((idx[a] >> p) & 1) << t;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      if (p < k) {
+#pragma unroll
+        for (int a = 0; a < A; ++a) {
+          const uint32_t w = __ballot_sync(0xffffffffu, (idx[a] >> p) & 1);
+          if (lane == p * A + a) *row_word = w;
+        }
+      }
+    }
+  }
+}
+
+// QJL projection of the residual held in shared memory (r_s[0..d_pad)):
+// lane l computes z_i for rows i = 32c + l and the sign words are formed by
+// ballot; lane c ends with sign word c in *sign_word (c < m/32).
+__device__ __forceinline__ void qjl_signs(const QParams& qp, const float* r_s, int lane,
+                                          uint32_t* sign_word) {
+  const int m = qp.m, dp = qp.d_pad;
+  for (int c0 = 0; c0 < m / 32; c0 += 4) {
+    float z[4] = {0.f, 0.f, 0.f, 0.f};
+    const int nc = min(4, m / 32 - c0);
+    for (int j = 0; j < dp; ++j) {
+      const float rj = r_s[j];
+      const float* st = qp.St + (size_t)j * m + (c0 * 32 + lane);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (u < nc) z[u] = fmaf(__ldg(st + u * 32), rj, z[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (u < nc) {
+        const uint32_t w = __ballot_sync(0xffffffffu, z[u] >= 0.0f);
+        if (lane == c0 + u) *sign_word = w;
+      }
+    }
+  }
+}
+
+// One warp task = up to 32 consecutive vectors of one segment (= one BLOCK32
+// block).  Grid-stride over tasks.
+template <int A, typename T, bool PROD>
+__global__ void __launch_bounds__(128) encode_hadamard_kernel(
+    QParams qp, const T* __restrict__ x, int64_t ld, int64_t seg_len, int64_t seg_cap,
+    int64_t blocks_per_seg, int64_t n_tasks, int layout, uint32_t* __restrict__ codes,
+    uint32_t* __restrict__ signs, float* __restrict__ norms, float* __restrict__ rnorms) {
+  __shared__ SmemCodebook cb;
+  __shared__ float r_s[4][PROD ? 32 * A : 1];
+  load_codebook(cb, qp);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const bool block_layout = layout == TQ_LAYOUT_BLOCK32;
+  const int k = qp.k;
+  const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib; task < n_tasks;
+       task += warps_total) {
+    const int64_t s = task / blocks_per_seg;
+    const int64_t b = task % blocks_per_seg;
+    const int nv = (int)min64(32, seg_len - 32 * b);
+    uint32_t blk[4][A];
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+      for (int a = 0; a < A; ++a) blk[p][a] = 0u;
+    for (int t = 0; t < nv; ++t) {
+      const int64_t row = s * seg_len + 32 * b + t;
+      const int64_t slot = s * seg_cap + 32 * b + t;
+      const T* xr = x + row * ld;
+      float v[A];
+      float ss = 0.f;
+#pragma unroll
+      for (int a = 0; a < A; ++a) {
+        const int j = 32 * a + lane;
+        v[a] = j < qp.d ? to_f32(xr[j]) : 0.0f;
+        ss = fmaf(v[a], v[a], ss);
+      }
+      ss = warp_sum(ss);
+      const float n = sqrtf(ss);
+      apply_signs<A>(v, qp.dmask, lane);
+      warp_fwht<A>(v, lane);
+      const float scale = n > 0.0f ? qp.inv_sqrt_dpad / n : 0.0f;
+#pragma unroll
+      for (int a = 0; a < A; ++a) v[a] *= scale;
+      int idx[A];
+      uint32_t row_word = 0;
+      quantize_pack<A>(v, idx, cb, k, lane, &row_word, blk, t, block_layout);
+      if (!block_layout && lane < k * A) codes[slot * qp.code_words + lane] = row_word;
+      if (lane == 0) norms[slot] = n;
+      if (PROD) {
+        float rr = 0.f;
+#pragma unroll
+        for (int a = 0; a < A; ++a) {
+          const float r = v[a] - cb.c[idx[a]];
+          rr = fmaf(r, r, rr);
+          r_s[wib][32 * a + lane] = r;
+        }
+        rr = warp_sum(rr);
+        __syncwarp();
+        uint32_t sw = 0;
+        qjl_signs(qp, r_s[wib], lane, &sw);
+        if (lane < qp.sign_words) signs[slot * qp.sign_words + lane] = sw;
+        if (lane == 0) rnorms[slot] = sqrtf(rr);
+        __syncwarp();
+      }
+    }
+    if (block_layout) {
+      uint32_t* dst = codes + (s * (seg_cap / 32) + b) * (int64_t)(k * 32 * A);
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        if (p < k)
+#pragma unroll
+          for (int a = 0; a < A; ++a) dst[p * 32 * A + 32 * a + lane] = blk[p][a];
+    }
+  }
+}
+
+// Dense path, step 1: n = ||x|| and x / n (fp32) for a chunk of vectors.
+template <typename T>
+__global__ void __launch_bounds__(128) normalize_rows_kernel(const T* __restrict__ x, int64_t ld,
+                                                             int d, int64_t seg_len,
+                                                             int64_t seg_cap, int64_t row0,
+                                                             int64_t nrows,
+                                                             float* __restrict__ xhat,
+                                                             float* __restrict__ norms) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (w >= nrows) return;
+  const int64_t row = row0 + w;
+  const T* xr = x + row * ld;
+  float ss = 0.f;
+  for (int j = lane; j < d; j += 32) {
+    const float v = to_f32(xr[j]);
+    ss = fmaf(v, v, ss);
+  }
+  ss = warp_sum(ss);
+  const float n = sqrtf(ss);
+  const float inv = n > 0.f ? 1.0f / n : 0.0f;
+  for (int j = lane; j < d; j += 32) xhat[w * d + j] = to_f32(xr[j]) * inv;
+  if (lane == 0) {
+    const int64_t s = row / seg_len, t = row % seg_len;
+    norms[s * seg_cap + t] = n;
+  }
+}
+
+// Dense path, step 3: quantize rotated rows y (fp32 [nrows][d]) and pack.
+// Q_prod also overwrites y with r = y - C[idx] and writes rho.  One warp
+// per 32-vector task; the host splits chunks at segment and block boundaries.
+__global__ void __launch_bounds__(128) quantize_rows_kernel(
+    QParams qp, float* __restrict__ y, int64_t seg_len, int64_t seg_cap, int64_t row0,
+    int64_t nrows, int layout, bool prod, uint32_t* __restrict__ codes,
+    float* __restrict__ rnorms) {
+  __shared__ SmemCodebook cb;
+  load_codebook(cb, qp);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const int k = qp.k, A = qp.d_pad / 32, d = qp.d;
+  const int nb = (1 << k) - 1;
+  const int64_t first = 32 * ((int64_t)blockIdx.x * 4 + wib);
+  if (first >= nrows) return;
+  const int nv = (int)min64(32, nrows - first);
+  const int64_t row = row0 + first;
+  const int64_t s = row / seg_len, t0 = row % seg_len;
+  if (layout == TQ_LAYOUT_BLOCK32) {
+    uint32_t* dst = codes + (s * (seg_cap / 32) + t0 / 32) * (int64_t)(k * 32 * A);
+    for (int a = 0; a < A; ++a) {
+      uint32_t blk[4] = {0u, 0u, 0u, 0u};
+      for (int t = 0; t < nv; ++t) {
+        const int idx = quantize_index(y[(first + t) * (int64_t)d + 32 * a + lane], cb.b, nb);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) blk[p] |= (uint32_t)((idx >> p) & 1) << t;
+      }
+      for (int p = 0; p < k; ++p) dst[p * 32 * A + 32 * a + lane] = blk[p];
+    }
+    return;
+  }
+  for (int t = 0; t < nv; ++t) {
+    float* yr = y + (first + t) * (int64_t)d;
+    const int64_t slot = s * seg_cap + t0 + t;
+    float rr = 0.f;
+    for (int a = 0; a < A; ++a) {
+      const float v = yr[32 * a + lane];
+      const int idx = quantize_index(v, cb.b, nb);
+      for (int p = 0; p < k; ++p) {
+        const uint32_t w = __ballot_sync(0xffffffffu, (idx >> p) & 1);
+        if (lane == 0) codes[slot * qp.code_words + p * A + a] = w;
+      }
+      if (prod) {
+        const float r = v - cb.c[idx];
+        rr = fmaf(r, r, rr);
+        yr[32 * a + lane] = r;
+      }
+    }
+    if (prod) {
+      rr = warp_sum(rr);
+      if (lane == 0) rnorms[slot] = sqrtf(rr);
+    }
+  }
+}
+
+// Dense path, step 5: sign bits of z = r S^T (fp32 [nrows][m]).
+__global__ void __launch_bounds__(128) pack_signs_kernel(const float* __restrict__ z, int m,
+                                                         int64_t seg_len, int64_t seg_cap,
+                                                         int64_t row0, int64_t nrows,
+                                                         uint32_t* __restrict__ signs) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (w >= nrows) return;
+  const int64_t row = row0 + w;
+  const int64_t slot = (row / seg_len) * seg_cap + row % seg_len;
+  for (int c = 0; c < m / 32; ++c) {
+    const uint32_t word = __ballot_sync(0xffffffffu, z[w * m + 32 * c + lane] >= 0.0f);
+    if (lane == 0) signs[slot * (m / 32) + c] = word;
+  }
+}
+
+}  // namespace tq
