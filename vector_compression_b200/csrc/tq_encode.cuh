@@ -64,10 +64,10 @@ __device__ __forceinline__ void quantize_pack(const float (&y)[A], int (&idx)[A]
 }
 
 // QJL projection of the residual held in shared memory (r_s[0..d_pad)):
-// lane l computes z_i for rows i = 32c + l and the sign words are formed by
-// ballot; lane c ends with sign word c in *sign_word (c < m/32).
+// lane l computes z_i for rows i = 32c + l; sign word c is the ballot of
+// z_i >= 0 over the warp and is written by lane 0 to dst[c].
 __device__ __forceinline__ void qjl_signs(const QParams& qp, const float* r_s, int lane,
-                                          uint32_t* sign_word) {
+                                          uint32_t* dst) {
   const int m = qp.m, dp = qp.d_pad;
   for (int c0 = 0; c0 < m / 32; c0 += 4) {
     float z[4] = {0.f, 0.f, 0.f, 0.f};
@@ -83,7 +83,7 @@ __device__ __forceinline__ void qjl_signs(const QParams& qp, const float* r_s, i
     for (int u = 0; u < 4; ++u) {
       if (u < nc) {
         const uint32_t w = __ballot_sync(0xffffffffu, z[u] >= 0.0f);
-        if (lane == c0 + u) *sign_word = w;
+        if (lane == 0) dst[c0 + u] = w;
       }
     }
   }
@@ -149,9 +149,7 @@ __global__ void __launch_bounds__(128) encode_hadamard_kernel(
         }
         rr = warp_sum(rr);
         __syncwarp();
-        uint32_t sw = 0;
-        qjl_signs(qp, r_s[wib], lane, &sw);
-        if (lane < qp.sign_words) signs[slot * qp.sign_words + lane] = sw;
+        qjl_signs(qp, r_s[wib], lane, signs + slot * qp.sign_words);
         if (lane == 0) rnorms[slot] = sqrtf(rr);
         __syncwarp();
       }
