@@ -61,7 +61,7 @@ def test_encode_mse_parity(d, dtype, layout, n, bits):
         if n % 32:
             assert np.all((tail >> np.uint32(n % 32)) == 0)
     check_codes(gi, e["idx"], e["y"], ora.boundaries, ora.d_pad)
-    gn = norms.cpu().numpy()
+    gn = norms.cpu().numpy()[:n]  # BLOCK32 keeps seg_cap (a multiple of 32) slots
     assert gn[min(5, n - 1)] == 0.0
     assert_close_rel(gn, e["norms"], 1e-30, what="norms")
 
@@ -268,7 +268,7 @@ def test_attention_end_to_end_qwen_shape_subset():
 def test_dense_rotation_encode_scores(bits):
     d = 256
     ora, lib = make_pair(d, bits, True, seed=50, dense=True)
-    _, pi, = lib.tables()[1:], lib.tables()[2]
+    pi = lib.tables()[2]
     assert np.max(np.abs(pi - ora.rot.Pi)) < 2e-7
     x = synth.gaussian_vectors(2000, d, seed=4, device=DEV, n_outliers=8, outlier_scale=10.0, normalize=True)
     q = synth.gaussian_vectors(16, d, seed=5, device=DEV, normalize=True)
