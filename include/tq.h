@@ -260,6 +260,41 @@ tq_status tq_decode_attention_workspace_size(const tq_params* kp, const tq_param
                                              size_t* bytes);
 
 /*
+ * tq_decode_attention_noalloc -- tq_decode_attention with no workspace
+ * argument and no allocation of any kind.  The pages have no counterpart to
+ * this call; it exists for deployment.
+ *
+ * Some callers cannot call cudaMalloc or otherwise obtain device memory on
+ * the decode path: for example a plugin inside an inference engine that owns
+ * every byte of the device's memory pool and offers plugins no allocation
+ * hook, or a latency-bound decode loop that must never risk the device-wide
+ * synchronization an allocation can cause.  This entry point serves them.
+ *
+ * Its scratch is one file-scope device array of TQ_NOALLOC_SCRATCH_BYTES
+ * (32 MiB), part of the library image: every GPU that loads libtq holds it
+ * until the process exits.  A call whose tq_decode_attention_workspace_size
+ * is larger returns TQ_ERR_WORKSPACE and enqueues nothing.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any
+ * stream capture.  Every call shares the same array.  The attention kernels
+ * overwrite every scratch byte they read, so nothing relies on its previous
+ * contents; but calls that overlap on the GPU (other streams, other host
+ * threads) race on the array and corrupt each other's results -- serialize
+ * them.
+ *
+ * Arguments, layouts, results and the other errors are those of
+ * tq_decode_attention.
+ */
+#define TQ_NOALLOC_SCRATCH_BYTES (32u << 20)
+tq_status tq_decode_attention_noalloc(const tq_params* kp, const tq_params* vp, const float* q,
+                                      int L, int B, int Hq, int Hkv, int64_t seq, int64_t cap,
+                                      float scale, const uint32_t* kcodes, const uint32_t* ksigns,
+                                      const float* knorms, const float* krnorms,
+                                      const uint32_t* vcodes, const float* vnorms, float* out,
+                                      void* stream);
+
+/*
  * tq_sync_check -- synchronize `stream` and report (then clear) the device
  * error word that kernels set when a bounded wait expires (TQ_ERR_TIMEOUT)
  * or an internal check fails (TQ_ERR_INTERNAL).

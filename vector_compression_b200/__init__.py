@@ -20,6 +20,7 @@ from ._lib import (BF16, F16, F32, LAYOUT_BLOCK32, LAYOUT_ROW, MODE_MSE, MODE_PR
 __all__ = [
     "TQParams", "tq_build_codebook", "tq_make_rotation", "tq_params_create", "tq_encode_mse", "tq_encode_prod",
     "tq_decode", "tq_scores", "tq_decode_attention", "tq_decode_attention_workspace_size",
+    "tq_decode_attention_noalloc",
     "tq_sync_check", "tq_version", "lib_path", "TQError",
 ]
 
@@ -257,6 +258,26 @@ def tq_decode_attention(kp: TQParams, vp: TQParams, q, kcache, vcache, seq: int,
         kp.handle, vp.handle, _ptr(qc), Ln, B, Hq, Hkv, seq, cap, float(scale),
         _ptr(kcodes), _ptr(ksigns), _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms),
         _ptr(out), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)))
+    return out
+
+
+def tq_decode_attention_noalloc(kp: TQParams, vp: TQParams, q, kcache, vcache, seq: int, cap: int,
+                                scale: float, out=None, stream=None):
+    """tq_decode_attention without a workspace: the library's fixed device
+    scratch array is used instead (see include/tq.h for its size limit and for
+    why overlapping calls must be serialized)."""
+    torch = _torch()
+    Ln, B, Hq, d = q.shape
+    kcodes, ksigns, knorms, krnorms = kcache
+    vcodes, vnorms = vcache
+    Hkv = knorms.numel() // (Ln * B * cap)
+    if out is None:
+        out = torch.empty((Ln, B, Hq, d), dtype=torch.float32, device=q.device)
+    qc = q.contiguous()
+    L.check("tq_decode_attention_noalloc", L.lib().tq_decode_attention_noalloc(
+        kp.handle, vp.handle, _ptr(qc), Ln, B, Hq, Hkv, seq, cap, float(scale),
+        _ptr(kcodes), _ptr(ksigns), _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms),
+        _ptr(out), _stream(stream)))
     return out
 
 
