@@ -5,16 +5,36 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 
 #include "tq_attention.cuh"
 #include "tq_device.cuh"
 #include "tq_encode.cuh"
+#include "tq_encode2.cuh"
+#include "tq_enc2_launch.h"
 #include "tq_gemm.cuh"
 #include "tq_internal.h"
 #include "tq_scores.cuh"
 
 namespace tq {
+
+// Error word set by kernels whose bounded waits expire; read and cleared by
+// tq_sync_check.  Kernels in other translation units get its address.
+__device__ unsigned int g_device_error = 0;
+
 namespace {
+
+unsigned* device_error_ptr() {
+  static unsigned* ptrs[128] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) ptrs[dev] = (unsigned*)p;
+  }
+  return ptrs[dev];
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
@@ -94,6 +114,77 @@ cudaError_t encode_dense(const QParams& qp, bool prod, const T* x, int64_t ld, i
 
 constexpr int64_t kDenseChunk = 32768;
 
+// ---------------------------------------------------------------- thread-per-vector encode
+
+// Returns true (and launches) when the thread-per-vector kernels cover the
+// request: Hadamard rotation, d_pad 128 or 256, 16-byte input rows and, for
+// Q_prod, m in {64, 128, 256}.
+bool try_encode_v2(const QParams& qp, bool prod, const void* x, int dt, int64_t n_vec, int64_t ld,
+                   int64_t seg_len, int64_t seg_cap, int layout, uint32_t* codes, uint32_t* signs,
+                   float* norms, float* rnorms, cudaStream_t st, cudaError_t* err) {
+  if (qp.rot != TQ_ROT_HADAMARD || (qp.d_pad != 128 && qp.d_pad != 256)) return false;
+  const int esz = (int)dtype_size(dt);
+  if ((qp.d * esz) % 16 != 0) return false;
+  if (prod && qp.m != 64 && qp.m != 128 && qp.m != 256) return false;
+  if (prod && qp.k > 3) return false;
+  enc2::SignMasks sg;
+  for (int j = 0; j < kMaxHadamard; ++j) sg.m[j] = 0;
+  auto dbit = [&](int j) { return (qp.dmask[j / 32] >> (j % 32)) & 1u; };
+  if (esz == 2) {
+    for (int p = 0; p < qp.d_pad / 2; ++p) sg.m[p] = (dbit(2 * p) << 15) | (dbit(2 * p + 1) << 31);
+  } else {
+    for (int j = 0; j < qp.d_pad; ++j) sg.m[j] = dbit(j) << 31;
+  }
+  enc2::Args a;
+  a.st.x = (const unsigned char*)x;
+  a.st.ld_bytes = ld * esz;
+  a.st.row_bytes = qp.d * esz;
+  const int cpr = a.st.row_bytes / 16;
+  a.st.pitch = (cpr + ((cpr % 2 == 0) ? 1 : 2)) * 16;
+  a.seg_len = seg_len;
+  a.seg_cap = seg_cap;
+  a.bps = ceil_div(seg_len, 32);
+  a.n_tasks = (n_vec / seg_len) * a.bps;
+  a.codes = codes;
+  a.signs = signs;
+  a.norms = norms;
+  a.rnorms = rnorms;
+  const size_t s_bytes = prod ? (size_t)qp.m * qp.d_pad * 2 : 0;
+  const size_t stage1 = (size_t)4 * 32 * a.st.pitch;
+  a.nbuf = (s_bytes + 2 * stage1 <= 113 * 1024) ? 2 : 1;
+  size_t smem = s_bytes + a.nbuf * stage1;
+  if (smem > 220 * 1024) return false;
+  int tmem_cols = 0;
+  if (prod) {
+    const int need = qp.d_pad + qp.m;
+    tmem_cols = 32;
+    while (tmem_cols < need) tmem_cols *= 2;
+    // at most 512 / tmem_cols CTAs may share an SM; pad shared memory so no
+    // more than that can be co-resident
+    const int per_sm = 512 / tmem_cols;
+    if (per_sm == 1 && smem < 120 * 1024) smem = 120 * 1024;
+  }
+  a.tmem_cols = tmem_cols;
+  if (a.n_tasks == 0) {
+    *err = cudaSuccess;
+    return true;
+  }
+  const int64_t want = ceil_div(a.n_tasks, 4);
+  const int resident = (smem <= 113 * 1024) ? 2 : 1;
+  const int ctas = (int)std::min<int64_t>(want, (int64_t)num_sms() * resident);
+  const int mode = prod ? enc2::MODE_PROD : (layout == TQ_LAYOUT_BLOCK32 ? enc2::MODE_MSE_BLOCK : enc2::MODE_MSE_ROW);
+  a.err = device_error_ptr();
+  if (!a.err) return false;
+  cudaError_t e;
+  switch (dt) {
+    case TQ_F32: e = enc2::launch_f32(qp.d_pad, mode, qp, sg, a, smem, ctas, st); break;
+    case TQ_F16: e = enc2::launch_f16(qp.d_pad, mode, qp, sg, a, smem, ctas, st); break;
+    default: e = enc2::launch_bf16(qp.d_pad, mode, qp, sg, a, smem, ctas, st); break;
+  }
+  *err = e;
+  return true;
+}
+
 size_t encode_workspace_bytes(const QParams& qp, bool prod, int64_t n_vec) {
   if (qp.rot != TQ_ROT_DENSE || n_vec == 0) return 0;
   const int64_t chunk = std::min<int64_t>(kDenseChunk, round_up(n_vec, 32));
@@ -102,11 +193,25 @@ size_t encode_workspace_bytes(const QParams& qp, bool prod, int64_t n_vec) {
 
 }  // namespace
 
+// The thread-per-vector encoder is used whenever it covers a request; the
+// environment variable TQ_ENCODE_V1=1 selects the warp-per-vector kernels
+// instead (kept as a second implementation for cross-checks).
+static const bool g_encode_v2 = [] {
+  const char* e = getenv("TQ_ENCODE_V1");
+  return !(e && e[0] == '1');
+}();
+
 int launch_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_vec, int64_t ld,
                   int64_t seg_len, int64_t seg_cap, int layout, uint32_t* codes, uint32_t* signs,
                   float* norms, float* rnorms, void* ws, void* stream) {
   const int64_t n_seg = n_vec / seg_len;
   cudaStream_t st = S(stream);
+  {
+    cudaError_t e2;
+    if (g_encode_v2 && try_encode_v2(qp, prod, x, dt, n_vec, ld, seg_len, seg_cap, layout, codes,
+                                     signs, norms, rnorms, st, &e2))
+      return e2;
+  }
   if (qp.rot == TQ_ROT_DENSE) {
     const int64_t chunk = std::min<int64_t>(kDenseChunk, round_up(n_vec, 32));
     float* w = (float*)ws;

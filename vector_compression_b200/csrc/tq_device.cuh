@@ -11,14 +11,6 @@
 
 namespace tq {
 
-// Error word set by kernels whose bounded waits expire or whose internal
-// checks fail; read and cleared by tq_sync_check.
-__device__ unsigned int g_device_error = 0;
-
-__device__ __forceinline__ void set_device_error(unsigned code) {
-  atomicCAS(&g_device_error, 0u, code);
-}
-
 template <typename T>
 __device__ __forceinline__ float to_f32(T v);
 template <>
