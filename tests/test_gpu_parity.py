@@ -231,7 +231,8 @@ def test_attention_on_oracle_cache(d, G, seq, cap, bits):
                 want = o.decode_attention(q[l, b, h * G:(h + 1) * G], kq, vq, ke, ve, scale, G)
                 got = out[l, b, h * G:(h + 1) * G]
                 err = np.linalg.norm(got - want, axis=1) / np.linalg.norm(want, axis=1)
-                assert err.max() <= 1e-5, err.max()
+                print(f"attention rel err (G={G}, bits={bits}): {err.max():.2e}")
+                assert err.max() <= REL_TOL, err.max()
 
 
 def test_attention_end_to_end_qwen_shape_subset():

@@ -8,6 +8,7 @@
 #include <cstdlib>
 
 #include "tq_attention.cuh"
+#include "tq_attn2.h"
 #include "tq_device.cuh"
 #include "tq_encode.cuh"
 #include "tq_encode2.cuh"
@@ -325,7 +326,7 @@ size_t attention_workspace(const QParams& kp, const QParams& vp, int L, int B, i
   const int G = Hq / Hkv;
   const int64_t target = (int64_t)num_sms() * 32;
   int64_t n_chunks = std::max<int64_t>(1, ceil_div(target, std::max<int64_t>(groups, 1)));
-  int64_t chunk = round_up(ceil_div(seq, n_chunks), 32);
+  int64_t chunk = round_up(ceil_div(seq, n_chunks), 64);
   chunk = std::max<int64_t>(chunk, 256);
   n_chunks = ceil_div(seq, chunk);
   if (chunk_out) *chunk_out = (int)chunk;
@@ -334,6 +335,19 @@ size_t attention_workspace(const QParams& kp, const QParams& vp, int L, int B, i
   size_t bytes = round_up((size_t)nq * kp.d_pad * 4, 256) + round_up((size_t)nq * kp.m * 4, 256) +
                  round_up((size_t)groups * n_chunks * G * (vp.d_pad + 2) * 4, 256);
   return bytes;
+}
+
+// The tensor-core kernel (tq_attn2.cu) covers d_pad = 128, m = 128, at most 8
+// query heads per KV head and key codes of 1..3 bits; TQ_ATTN_V1=1 selects
+// the SIMT kernel for every shape.
+static const bool g_attn_v2 = [] {
+  const char* e = getenv("TQ_ATTN_V1");
+  return !(e && e[0] == '1');
+}();
+
+static bool attn2_covers(const QParams& kp, const QParams& vp, int G) {
+  return g_attn_v2 && kp.rot == TQ_ROT_HADAMARD && kp.d_pad == 128 && vp.d_pad == 128 &&
+         kp.m == 128 && G >= 1 && G <= 8 && kp.k >= 1 && kp.k <= 3 && vp.k >= 1 && vp.k <= 4;
 }
 
 int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q, int L, int B,
@@ -361,6 +375,29 @@ int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q
   sh.seq = seq;
   sh.cap = cap;
   sh.scale = scale;
+  if (attn2_covers(kp, vp, sh.G)) {
+    attn2::Params p2;
+    p2.G = sh.G;
+    p2.chunk = chunk;
+    p2.n_chunks = n_chunks;
+    p2.seq = seq;
+    p2.cap = cap;
+    p2.scale = scale;
+    p2.kappa = kp.kappa;
+    p2.qrot = qrot;
+    p2.u = u;
+    p2.kcodes = kcodes;
+    p2.ksigns = ksigns;
+    p2.knorms = knorms;
+    p2.krnorms = krnorms;
+    p2.vcodes = vcodes;
+    p2.vnorms = vnorms;
+    p2.part = part;
+    attn2::odd_feature_coefs(kp.centroids, kp.k, p2.kalpha, &p2.kalpha_sum);
+    attn2::odd_feature_coefs(vp.centroids, vp.k, p2.valpha, &p2.valpha_sum);
+    cudaError_t ce = attn2::launch(p2, kp.k, vp.k, dim3((unsigned)n_chunks, (unsigned)sh.groups), st);
+    if (ce != cudaSuccess) return ce;
+  } else {
   const size_t smem = (size_t)sh.G * (kp.d_pad + kp.m) * sizeof(float);
   static bool attr_set = false;
   if (!attr_set) {
@@ -375,6 +412,7 @@ int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q
     attention_chunk_kernel<2><<<grid, kAttnThreads, smem, st>>>(kp, vp, sh, qrot, u, kcodes, ksigns, knorms, krnorms, vcodes, vnorms, part);
   cudaError_t ce = cudaGetLastError();
   if (ce != cudaSuccess) return ce;
+  }
   const unsigned cblocks = (unsigned)ceil_div((int64_t)sh.groups * sh.G, 4);
   switch (vp.d_pad / 32) {
 #define TQ_CMB(AA)                                                                                 \

@@ -418,3 +418,58 @@ tq_status tq_params_tables(const tq_params* p, float* centroids, float* boundari
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ attention feature coefficients
+
+#include "tq_attn2.h"
+
+namespace tq {
+namespace attn2 {
+
+void odd_feature_coefs(const float* centroids, int k, float* alpha, float* alpha_sum) {
+  // subsets as bit masks in the kernel's order
+  int subsets[8];
+  int nf = 0;
+  for (int p = 0; p < k; ++p) subsets[nf++] = 1 << p;
+  if (k == 3) subsets[nf++] = 0x7;
+  if (k == 4) {
+    for (int t = 0; t < 4; ++t) subsets[nf++] = 0xF & ~(1 << (3 - t));
+  }
+  const int n = 1 << (k - 1);
+  // rows: idx = n + mu (upper half); columns: features
+  double A[8][9];
+  for (int r = 0; r < n; ++r) {
+    const int idx = n + r;
+    for (int f = 0; f < nf; ++f) {
+      double v = 1.0;
+      for (int p = 0; p < k; ++p)
+        if (subsets[f] & (1 << p)) v *= ((idx >> p) & 1) ? 1.0 : -1.0;
+      A[r][f] = v;
+    }
+    A[r][nf] = centroids[idx];
+  }
+  // Gauss-Jordan elimination with partial pivoting (n <= 8)
+  for (int col = 0; col < n; ++col) {
+    int piv = col;
+    for (int r = col + 1; r < n; ++r)
+      if (std::fabs(A[r][col]) > std::fabs(A[piv][col])) piv = r;
+    for (int j = 0; j <= n; ++j) std::swap(A[col][j], A[piv][j]);
+    const double d = A[col][col];
+    for (int j = 0; j <= n; ++j) A[col][j] /= d;
+    for (int r = 0; r < n; ++r) {
+      if (r == col) continue;
+      const double f = A[r][col];
+      for (int j = 0; j <= n; ++j) A[r][j] -= f * A[col][j];
+    }
+  }
+  double s = 0.0;
+  for (int f = 0; f < 8; ++f) alpha[f] = 0.f;
+  for (int f = 0; f < n; ++f) {
+    alpha[f] = (float)A[f][n];
+    s += A[f][n];
+  }
+  *alpha_sum = (float)s;
+}
+
+}  // namespace attn2
+}  // namespace tq
