@@ -5,6 +5,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdio>
 #include <cstdlib>
 
 #include "tq_attention.cuh"
@@ -13,6 +14,7 @@
 #include "tq_encode.cuh"
 #include "tq_encode2.cuh"
 #include "tq_enc2_launch.h"
+#include "tq_enc3.h"
 #include "tq_gemm.cuh"
 #include "tq_internal.h"
 #include "tq_scores.cuh"
@@ -194,12 +196,17 @@ size_t encode_workspace_bytes(const QParams& qp, bool prod, int64_t n_vec) {
 
 }  // namespace
 
-// The thread-per-vector encoder is used whenever it covers a request; the
-// environment variable TQ_ENCODE_V1=1 selects the warp-per-vector kernels
-// instead (kept as a second implementation for cross-checks).
+// Encoder selection: the tensor-core encoder whenever it covers a request,
+// else the thread-per-vector one, else the warp-per-vector kernels.  The
+// environment variable TQ_ENCODE_V2=1 skips the first, TQ_ENCODE_V1=1 both
+// (the older kernels stay as second implementations for cross-checks).
 static const bool g_encode_v2 = [] {
   const char* e = getenv("TQ_ENCODE_V1");
   return !(e && e[0] == '1');
+}();
+static const bool g_encode_tc = [] {
+  const char* e = getenv("TQ_ENCODE_V2");
+  return g_encode_v2 && !(e && e[0] == '1');
 }();
 
 int launch_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_vec, int64_t ld,
@@ -209,6 +216,9 @@ int launch_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n
   cudaStream_t st = S(stream);
   {
     cudaError_t e2;
+    if (g_encode_tc && enc3::try_encode(qp, prod, x, dt, n_vec, ld, seg_len, seg_cap, layout, codes,
+                                        signs, norms, rnorms, device_error_ptr(), num_sms(), st, &e2))
+      return e2;
     if (g_encode_v2 && try_encode_v2(qp, prod, x, dt, n_vec, ld, seg_len, seg_cap, layout, codes,
                                      signs, norms, rnorms, st, &e2))
       return e2;
@@ -448,7 +458,16 @@ int read_and_clear_device_error(void* stream, unsigned* err) {
 
 namespace {
 
-tq_status cuda_status(int e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
+// With TQ_VERBOSE=1 in the environment, CUDA failures are also named on stderr.
+tq_status cuda_status(int e) {
+  if (e == cudaSuccess) return TQ_OK;
+  static const bool verbose = [] {
+    const char* v = getenv("TQ_VERBOSE");
+    return v && v[0] == '1';
+  }();
+  if (verbose) fprintf(stderr, "libtq: CUDA error %d (%s)\n", e, cudaGetErrorName((cudaError_t)e));
+  return TQ_ERR_CUDA;
+}
 
 tq_status check_segments(int64_t n_vec, int64_t* seg_len, int64_t* seg_cap, bool block) {
   if (n_vec < 0) return TQ_ERR_INVALID_ARG;

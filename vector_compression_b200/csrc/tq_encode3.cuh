@@ -1,0 +1,593 @@
+// Encode kernels with the rotation on the tensor cores (d_pad = 128, fp16 or
+// bf16 input, randomized Hadamard rotation).
+//
+// Same method as the other encoders (TurboQuant blog notes, Q_MSE and the
+// definition of Q_prod; explainer §6, §8): n = ||x||, y = H D x / (sqrt(d_pad) n),
+// idx = #{k : B_k < y}, bit-packed codes; Q_prod adds r = y - C[idx],
+// rho = ||r|| and the sign bits of S r.
+//
+// The randomized Hadamard rotation is the product with the d_pad x d_pad
+// matrix H D, whose entries are +-1: exact in fp16 and bf16.  One tcgen05 MMA
+// per tile of 128 vectors computes u = (H D) x for all of them with exact
+// products and fp32 accumulation, so the CUDA cores are left with the
+// per-coordinate quantization only.  Roles inside a persistent CTA (one per SM):
+//   warp 0      TMA producer: tiles of 128 consecutive input rows, two
+//               128-byte-swizzled boxes of 64 columns each, into a 4-stage ring;
+//   warp 1      TMEM allocator and MMA issuer (one elected thread);
+//   warps 2..9  two epilogue groups of four warps; group g owns TMEM buffer g
+//               and every second tile.  Thread (warp w, lane l) reads TMEM lane
+//               32 (w % 4) + l, i.e. one vector: its 128 values of u, the norm
+//               n = ||u|| / sqrt(d_pad), the sign plane and the binary search of
+//               |u| against the positive boundaries scaled by ||u||.
+// Q_prod: the epilogue writes r = u / ||u|| - C[idx] (times 2^10, split into fp16
+// hi + lo parts) back into its TMEM lane, a second MMA forms S r for the tile
+// (A = r from TMEM, B = S from shared memory) and the epilogue reads its row to
+// form the QJL sign words.
+// Exact boundary ties on the negative side resolve toward zero here (the
+// oracle resolves them to the lower cell); such values lie inside the parity
+// window by definition.
+//
+// Requirements checked by the host: rows are 16-byte aligned (d * 2 and the
+// row stride multiples of 16 bytes), every segment holds a multiple of 32
+// vectors (so each warp's 32 rows are one BLOCK32 block of one segment), and
+// m <= 128 for Q_prod.  Every wait is bounded; on expiry the device error word
+// is set and the CTA winds down.
+#pragma once
+
+#include <cuda.h>
+
+#include <type_traits>
+
+#include "tq_device.cuh"
+#include "tq_enc3.h"
+
+namespace tq {
+namespace enc3 {
+
+// ------------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+// Bounded wait for the phase with the given parity: false (and the device
+// error word set) if it has not completed within ~2^31 cycles.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (clock64() - t0 > (1LL << 31)) {
+      atomicCAS(err, 0u, (unsigned)TQ_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Warp-uniform form: every lane waits, the warp proceeds only if all saw it.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, unsigned* err) {
+  const bool ok = mbar_wait(bar, parity, err);
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// D (TMEM) (+)= A (smem descriptor) * B (smem descriptor)^T
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc));
+}
+// D (TMEM) (+)= A (TMEM) * B (smem descriptor)^T
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc));
+}
+
+// Shared-memory matrix descriptors (K-major operands).
+//  * no swizzle: 8x8 core matrices of 128 contiguous bytes, LBO = stride between
+//    core matrices along K, SBO = stride between 8-row groups;
+//  * 128-byte swizzle (what TMA writes for a box 64 x 16-bit wide): rows of
+//    128 bytes, 8-row groups 1024 bytes apart, chunks XOR-permuted by row.
+__device__ __forceinline__ uint64_t desc_noswz(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Byte offset of element (row, k) in a no-swizzle K-major tile of `rows` rows.
+__device__ __forceinline__ uint32_t core_offset(int row, int k, int rows) {
+  return (uint32_t)(((k >> 3) * (rows >> 3) + (row >> 3)) * 128 + (row & 7) * 16 + (k & 7) * 2);
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(addr));
+}
+
+// Completes outstanding tcgen05.ld of this thread; the empty asm statements
+// keep every use of the loaded registers after the wait.
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[N][32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int a = 0; a < N; ++a)
+#pragma unroll
+    for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[a][i]));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(addr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// ------------------------------------------------------------------ quantize + pack
+
+// 0xFFFFFFFF if a > b else 0 (an integer mask instead of a predicate).
+__device__ __forceinline__ uint32_t gt_mask(float a, float b) {
+  uint32_t r;
+  asm("set.gt.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+  return r;
+}
+// m ? a : b for an all-ones / all-zeros mask m
+__device__ __forceinline__ float sel_mask(uint32_t m, float a, float b) {
+  return __uint_as_float((m & __float_as_uint(a)) | (~m & __float_as_uint(b)));
+}
+
+// Quantize 32 coordinates u[0..32) (coordinate 32c + i in u[i]) against the
+// positive thresholds t (boundaries times ||u||) and shift the bit planes into
+// words (bit i = coordinate 32c + i): the sign plane S = [u > 0] and the
+// magnitude bits M of the binary search of |u|; the planes of
+// idx = s ? 2^(K-1) + mu : 2^(K-1) - 1 - mu are the top plane S and the lower
+// planes ~(S ^ M).  With RESID, u[i] becomes 2^10 r = u * inv - 2^10 C[idx]
+// (inv = 2^10 / ||u||, c = 2^10 times the positive centroids) and rr
+// accumulates its square.
+template <int K, bool RESID>
+__device__ __forceinline__ void quant32(float (&u)[32], const float (&t)[8], const float (&c)[8],
+                                        float inv, uint32_t (&plane)[K], float& rr) {
+  uint32_t S = 0, M0 = 0, M1 = 0, M2 = 0;
+#pragma unroll
+  for (int i = 31; i >= 0; --i) {
+    const float y = u[i];
+    const float a = fabsf(y);
+    const uint32_t s = gt_mask(y, 0.0f);
+    S = S + S - s;
+    float cm = c[0];
+    if (K == 2) {
+      const uint32_t m0 = gt_mask(a, t[0]);
+      M0 = M0 + M0 - m0;
+      if (RESID) cm = sel_mask(m0, c[1], c[0]);
+    } else if (K == 3) {
+      const uint32_t m1 = gt_mask(a, t[1]);
+      const uint32_t m0 = gt_mask(a, sel_mask(m1, t[2], t[0]));
+      M1 = M1 + M1 - m1;
+      M0 = M0 + M0 - m0;
+      if (RESID) cm = sel_mask(m1, sel_mask(m0, c[3], c[2]), sel_mask(m0, c[1], c[0]));
+    } else if (K == 4) {
+      const uint32_t m2 = gt_mask(a, t[3]);
+      const uint32_t m1 = gt_mask(a, sel_mask(m2, t[5], t[1]));
+      const float tA = sel_mask(m2, t[6], t[2]), tB = sel_mask(m2, t[4], t[0]);
+      const uint32_t m0 = gt_mask(a, sel_mask(m1, tA, tB));
+      M2 = M2 + M2 - m2;
+      M1 = M1 + M1 - m1;
+      M0 = M0 + M0 - m0;
+    }
+    if (RESID) {
+      // u * inv - C[idx], C[idx] = +cm for u > 0 and -cm otherwise
+      const float negc = __uint_as_float(__float_as_uint(cm) ^ (s & 0x80000000u));
+      const float r = fmaf(y, inv, negc);
+      u[i] = r;
+      rr = fmaf(r, r, rr);
+    }
+  }
+  plane[K - 1] = S;
+  if (K >= 2) plane[0] = ~(S ^ M0);
+  if (K >= 3) plane[1] = ~(S ^ M1);
+  if (K >= 4) plane[2] = ~(S ^ M2);
+}
+
+// 32x32 bit transpose across the warp: lane t holds row t (bit i); returns
+// column `lane` (bit t = row t's bit `lane`).
+struct TransposeCtl {
+  uint32_t keep[5];
+  uint32_t amt[5];
+};
+
+__device__ __forceinline__ TransposeCtl make_transpose_ctl(int lane) {
+  const uint32_t low[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+  TransposeCtl c;
+#pragma unroll
+  for (int r = 0; r < 5; ++r) {
+    const int s = 16 >> r;
+    const bool hi = (lane & s) != 0;
+    c.keep[r] = hi ? ~low[r] : low[r];
+    c.amt[r] = hi ? (uint32_t)(32 - s) : (uint32_t)s;
+  }
+  return c;
+}
+
+__device__ __forceinline__ uint32_t transpose32(uint32_t w, const TransposeCtl& c) {
+#pragma unroll
+  for (int r = 0; r < 5; ++r) {
+    const int s = 16 >> r;
+    const uint32_t o = __shfl_xor_sync(0xffffffffu, w, s);
+    const uint32_t rot = __funnelshift_l(o, o, c.amt[r]);
+    w = (w & c.keep[r]) | (rot & ~c.keep[r]);
+  }
+  return w;
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <typename T, int K, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, QParams qp, Args a) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages];
+  __shared__ __align__(8) uint64_t bar_accf[2], bar_acce[2], bar_aready[2], bar_zf[2], bar_done;
+  __shared__ uint32_t tmem_base_s;
+  constexpr bool PROD = MODE == MODE_PROD;
+  constexpr bool BF16 = sizeof(T) == 2 && !std::is_same<T, __half>::value;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m = qp.m;
+  // 1024-byte alignment for the swizzled tiles
+  unsigned char* smem =
+      smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  unsigned char* rot = smem;
+  unsigned char* smat = smem + kRotBytes;
+  unsigned char* stages = smat + (PROD ? m * kDP * 2 : 0);
+  const uint32_t tmem_cols = PROD ? 512u : 256u;
+  const uint32_t buf_cols = PROD ? 256u : 128u;
+
+  // ---- setup: rotation operand B[n][k] = H[n][k] D_k (+-1) and S, barriers, TMEM
+  {
+    const uint16_t one = BF16 ? 0x3F80u : 0x3C00u;
+    for (int e = tid; e < kDP * (kDP / 8); e += kThreads) {
+      const int n = e / (kDP / 8), kc = e % (kDP / 8);
+      uint16_t v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int k = kc * 8 + i;
+        const uint32_t neg = (__popc(n & k) & 1) ^ ((qp.dmask[k >> 5] >> (k & 31)) & 1u);
+        v[i] = (uint16_t)(one | (neg << 15));
+      }
+      uint4 w;
+      w.x = v[0] | ((uint32_t)v[1] << 16);
+      w.y = v[2] | ((uint32_t)v[3] << 16);
+      w.z = v[4] | ((uint32_t)v[5] << 16);
+      w.w = v[6] | ((uint32_t)v[7] << 16);
+      *reinterpret_cast<uint4*>(rot + core_offset(n, kc * 8, kDP)) = w;
+    }
+    if (PROD) {
+      for (int e = tid; e < m * (kDP / 8); e += kThreads) {
+        const int row = e / (kDP / 8), kc = e % (kDP / 8);
+        const uint4 w = *reinterpret_cast<const uint4*>(qp.S16 + (size_t)row * kDP + kc * 8);
+        *reinterpret_cast<uint4*>(smat + core_offset(row, kc * 8, m)) = w;
+      }
+    }
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&bar_full[s]), 1);
+      mbar_init(smem_u32(&bar_empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bar_accf[b]), 1);
+      mbar_init(smem_u32(&bar_acce[b]), 4);
+      mbar_init(smem_u32(&bar_aready[b]), 4);
+      mbar_init(smem_u32(&bar_zf[b]), 1);
+    }
+    mbar_init(smem_u32(&bar_done), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_base_s)),
+                 "r"(tmem_cols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  const int64_t G = gridDim.x;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int L = 0;; ++L) {
+        const int64_t tile = blockIdx.x + (int64_t)L * G;
+        if (tile >= a.n_tiles) break;
+        const int s = L % kStages;
+        if (L >= kStages && !mbar_wait(smem_u32(&bar_empty[s]), ((L / kStages) - 1) & 1, a.err)) break;
+        const uint32_t dst = smem_u32(stages + s * kTileBytes);
+        mbar_arrive_tx(smem_u32(&bar_full[s]), kTileBytes);
+        tma_load_2d(dst, &xmap, 0, (int)(tile * kRows), smem_u32(&bar_full[s]));
+        tma_load_2d(dst + kTileBytes / 2, &xmap, 64, (int)(tile * kRows), smem_u32(&bar_full[s]));
+        issued = L + 1;
+      }
+      // no copy may still be landing when the CTA exits
+      for (int L = issued - kStages < 0 ? 0 : issued - kStages; L < issued; ++L)
+        mbar_wait(smem_u32(&bar_full[L % kStages]), (L / kStages) & 1, a.err);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t fmt = BF16 ? 1u : 0u;
+      const uint32_t idesc1 = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kDP >> 3) << 17) |
+                              ((uint32_t)(kRows >> 4) << 24);
+      const uint32_t idesc2 =
+          (1u << 4) | ((uint32_t)(m >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
+      const uint32_t rot_base = smem_u32(rot);
+      const uint32_t s_base = smem_u32(smat);
+      const uint32_t s_lbo = (uint32_t)(m / 8) * 128u;
+      bool ok = true;
+      int L = 0;
+      for (;; ++L) {
+        const int64_t tile = blockIdx.x + (int64_t)L * G;
+        const bool have = tile < a.n_tiles;
+        if (have) {
+          const int s = L % kStages, b = L & 1;
+          if (!mbar_wait(smem_u32(&bar_full[s]), (L / kStages) & 1, a.err)) { ok = false; break; }
+          if (L >= 2 && !mbar_wait(smem_u32(&bar_acce[b]), ((L >> 1) - 1) & 1, a.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(stages + s * kTileBytes);
+          const uint32_t d_tmem = tmem + (uint32_t)b * buf_cols;
+#pragma unroll
+          for (int t = 0; t < kDP / 16; ++t) {
+            const uint64_t ad = desc_sw128(a_base + (uint32_t)(t >> 2) * (kTileBytes / 2) + (uint32_t)(t & 3) * 32u);
+            const uint64_t bd = desc_noswz(rot_base + (uint32_t)(2 * t) * 2048u, 2048u, 128u);
+            mma_ss(d_tmem, ad, bd, idesc1, t > 0 ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&bar_empty[s]));
+          tc_commit(smem_u32(&bar_accf[b]));
+        }
+        if (PROD && L >= 1) {
+          // S r for the previous tile, once its epilogue has written r
+          const int Lp = L - 1, b = Lp & 1;
+          if (!mbar_wait(smem_u32(&bar_aready[b]), (Lp >> 1) & 1, a.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_tmem = tmem + (uint32_t)b * buf_cols;
+          const uint32_t z_tmem = a_tmem + 128u;
+#pragma unroll
+          for (int pass = 0; pass < 2; ++pass) {  // hi, then lo parts of r
+#pragma unroll
+            for (int t = 0; t < kDP / 16; ++t) {
+              const uint32_t acol = (uint32_t)(32 * (t >> 1) + 16 * pass + 8 * (t & 1));
+              const uint64_t bd = desc_noswz(s_base + (uint32_t)(2 * t) * s_lbo, s_lbo, 128u);
+              mma_ts(z_tmem, a_tmem + acol, bd, idesc2, (pass | t) ? 1u : 0u);
+            }
+          }
+          tc_commit(smem_u32(&bar_zf[b]));
+        }
+        if (!have) break;
+      }
+      // every MMA issued above has completed before TMEM is released
+      tc_commit(smem_u32(&bar_done));
+      mbar_wait(smem_u32(&bar_done), 0, a.err);
+      (void)ok;
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int ew = warp - 2;          // 0..7
+    const int grp = ew >> 2;          // TMEM buffer / tile parity
+    const int quarter = warp & 3;     // TMEM lanes 32*quarter .. +31
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t ubase = tmem + (uint32_t)grp * buf_cols + lane_off;
+    const TransposeCtl tctl = make_transpose_ctl(lane);
+    const int half_levels = 1 << (K - 1);
+    float bpos[8], c1024[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      bpos[i] = i < half_levels - 1 ? qp.boundaries[half_levels + i] : 0.f;
+      c1024[i] = i < half_levels ? 1024.0f * qp.centroids[half_levels + i] : 0.f;
+    }
+    for (int L = grp;; L += 2) {
+      const int64_t tile = blockIdx.x + (int64_t)L * G;
+      if (tile >= a.n_tiles) break;
+      const uint32_t par = (uint32_t)(L >> 1) & 1u;
+      if (!mbar_wait_warp(smem_u32(&bar_accf[grp]), par, a.err)) break;
+      tc_fence_after();
+      const int64_t row = tile * kRows + quarter * 32 + lane;
+      const bool valid = row < a.n_vec;
+      const bool have = tile * kRows + quarter * 32 < a.n_vec;  // any valid row in this warp
+      const int64_t seg = valid ? row / a.seg_len : 0;
+      const int64_t pos = valid ? row - seg * a.seg_len : 0;
+      const int64_t slot = seg * a.seg_cap + pos;
+      // BLOCK32: the warp's 32 rows are one block of one segment (segments hold
+      // a multiple of 32 vectors and tiles start at multiples of 128 rows)
+      uint32_t* blk = nullptr;
+      if (MODE == MODE_MSE_BLOCK) {
+        const int64_t row0 = tile * kRows + quarter * 32;
+        const int64_t seg0 = row0 / a.seg_len;
+        blk = a.codes + (seg0 * (a.seg_cap / 32) + (row0 - seg0 * a.seg_len) / 32) * (int64_t)(K * kDP);
+      }
+
+      // pass 1: ||u|| over column chunks {0, 1} then {2, 3} (32 columns each);
+      // chunks 2 and 3 stay in registers for pass 2
+      uint32_t ur[2][32];
+      float ss0 = 0.f, ss1 = 0.f, ss2 = 0.f, ss3 = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        tmem_ld32(ubase + (uint32_t)(64 * h), ur[0]);
+        tmem_ld32(ubase + (uint32_t)(64 * h + 32), ur[1]);
+        tmem_ld_wait<2>(ur);
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float v0 = __uint_as_float(ur[c][i]), v1 = __uint_as_float(ur[c][i + 1]);
+            const float v2 = __uint_as_float(ur[c][i + 2]), v3 = __uint_as_float(ur[c][i + 3]);
+            ss0 = fmaf(v0, v0, ss0);
+            ss1 = fmaf(v1, v1, ss1);
+            ss2 = fmaf(v2, v2, ss2);
+            ss3 = fmaf(v3, v3, ss3);
+          }
+      }
+      const float nu = sqrtf((ss0 + ss1) + (ss2 + ss3));  // ||u|| = sqrt(d_pad) ||x||
+      if (valid) a.norms[slot] = nu * qp.inv_sqrt_dpad;
+      float th[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) th[i] = bpos[i] * nu;
+      const float inv = nu > 0.f ? 1024.0f / nu : 0.f;
+      float rr = 0.f;
+      uint32_t rowq[K][4];
+      // pass 2: chunks 2 and 3 from registers, then chunks 0 and 1 again
+#pragma unroll
+      for (int h = 1; h >= 0; --h) {
+        if (h == 0) {
+          tmem_ld32(ubase, ur[0]);
+          tmem_ld32(ubase + 32u, ur[1]);
+          tmem_ld_wait<2>(ur);
+          if (!PROD) {
+            // u has been read: the buffer is free for the next tile
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar_acce[grp]));
+          }
+        }
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * h + cc;
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ur[cc][i]);
+          uint32_t planes[K];
+          quant32<K, PROD>(v, th, c1024, inv, planes, rr);
+          if (MODE == MODE_MSE_BLOCK) {
+#pragma unroll
+            for (int p = 0; p < K; ++p) {
+              const uint32_t word = transpose32(valid ? planes[p] : 0u, tctl);
+              if (have) blk[p * kDP + 32 * c + lane] = word;
+            }
+          } else {
+#pragma unroll
+            for (int p = 0; p < K; ++p) rowq[p][c] = planes[p];
+          }
+          if (PROD) {
+            // this chunk's residual as fp16 hi (columns 32c .. 32c+15) and lo
+            // (32c+16 .. 32c+31) parts: |r| <= 2 so 2^10 r stays below the fp16
+            // maximum and its lo part out of the subnormal range; the sign of S r
+            // is unchanged by the scale.
+            uint32_t hiw[16], low[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const float r0 = v[2 * q], r1 = v[2 * q + 1];
+              const __half2 hv = __floats2half2_rn(r0, r1);
+              const float2 hf = __half22float2(hv);
+              const __half2 l = __floats2half2_rn(r0 - hf.x, r1 - hf.y);
+              hiw[q] = *reinterpret_cast<const uint32_t*>(&hv);
+              low[q] = *reinterpret_cast<const uint32_t*>(&l);
+            }
+            tmem_st16(ubase + (uint32_t)(32 * c), hiw);
+            tmem_st16(ubase + (uint32_t)(32 * c + 16), low);
+          }
+        }
+      }
+      if (MODE != MODE_MSE_BLOCK && valid) {
+        uint4* dst = reinterpret_cast<uint4*>(a.codes + slot * (int64_t)(K * 4));
+#pragma unroll
+        for (int p = 0; p < K; ++p) dst[p] = make_uint4(rowq[p][0], rowq[p][1], rowq[p][2], rowq[p][3]);
+      }
+      if (PROD) {
+        if (valid) a.rnorms[slot] = sqrtf(rr) * (1.0f / 1024.0f);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_aready[grp]));
+        if (!mbar_wait_warp(smem_u32(&bar_zf[grp]), par, a.err)) break;
+        tc_fence_after();
+        const uint32_t zbase = ubase + 128u;
+        uint32_t sw[8];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (32 * c < m) {
+            uint32_t z[1][32];
+            tmem_ld32(zbase + (uint32_t)(32 * c), z[0]);
+            tmem_ld_wait<1>(z);
+            uint32_t neg = 0;
+#pragma unroll
+            for (int i = 31; i >= 0; --i) neg = (neg << 1) | (z[0][i] >> 31);
+            sw[c] = ~neg;  // bit i = [ (S r)_(32c+i) >= 0 ]
+          } else {
+            sw[c] = 0u;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_acce[grp]));
+        if (valid) {
+          if (m == 128)
+            *reinterpret_cast<uint4*>(a.signs + slot * 4) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+          else
+            *reinterpret_cast<uint2*>(a.signs + slot * 2) = make_uint2(sw[0], sw[1]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols));
+  }
+}
+
+}  // namespace enc3
+}  // namespace tq
