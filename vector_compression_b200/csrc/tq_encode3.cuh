@@ -155,15 +155,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&r)[32]) {
       : "r"(addr));
 }
 
-// Completes outstanding tcgen05.ld of this thread; the empty asm statements
-// keep every use of the loaded registers after the wait.
-template <int N>
-__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[N][32]) {
+// Complete the outstanding tcgen05.ld of this thread; the empty asm
+// statements keep every use of the loaded registers after the wait.
+__device__ __forceinline__ void tmem_ld_wait1(uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int a = 0; a < N; ++a)
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
+}
+__device__ __forceinline__ void tmem_ld_wait2(uint32_t (&r)[32], uint32_t (&q)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[a][i]));
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]), "+r"(q[i]));
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t addr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(addr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t (&r)[16]) {
@@ -187,36 +195,66 @@ __device__ __forceinline__ float sel_mask(uint32_t m, float a, float b) {
   return __uint_as_float((m & __float_as_uint(a)) | (~m & __float_as_uint(b)));
 }
 
-// Quantize 32 coordinates u[0..32) (coordinate 32c + i in u[i]) against the
-// positive thresholds t (boundaries times ||u||) and shift the bit planes into
-// words (bit i = coordinate 32c + i): the sign plane S = [u > 0] and the
-// magnitude bits M of the binary search of |u|; the planes of
-// idx = s ? 2^(K-1) + mu : 2^(K-1) - 1 - mu are the top plane S and the lower
-// planes ~(S ^ M).  With RESID, u[i] becomes 2^10 r = u * inv - 2^10 C[idx]
-// (inv = 2^10 / ||u||, c = 2^10 times the positive centroids) and rr
-// accumulates its square.
-template <int K, bool RESID>
-__device__ __forceinline__ void quant32(float (&u)[32], const float (&t)[8], const float (&c)[8],
-                                        float inv, uint32_t (&plane)[K], float& rr) {
+// Sign bit of a - b.  The sign of a rounded difference is the sign of the
+// exact one and equal operands give +0, so for b = |u| and a = t the bit is
+// exactly [|u| > t]; for a = 0 and b = u it is [u > 0].
+__device__ __forceinline__ uint32_t sub_bits(float a, float b) {
+  float r;
+  asm("sub.rn.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return __float_as_uint(r);
+}
+// w << 1 with the sign bit of v shifted in at bit 0
+__device__ __forceinline__ uint32_t shift_in(uint32_t w, uint32_t v) { return __funnelshift_l(v, w, 1); }
+// 1.0 if v < 0 else 0.0, for |v| >= 2^-40 or v = +0
+__device__ __forceinline__ float step_neg(float v) {
+  float r;
+  asm("mul.rn.sat.f32 %0, %1, 0fD3800000;" : "=f"(r) : "f"(v));  // v * -2^40, clamped to [0, 1]
+  return r;
+}
+
+// Planes of idx = s ? 2^(K-1) + mu : 2^(K-1) - 1 - mu from the sign plane S
+// and the magnitude bits M of mu: the top plane is S, the lower ones ~(S ^ M).
+template <int K>
+__device__ __forceinline__ void planes_from(uint32_t S, uint32_t M0, uint32_t M1, uint32_t M2,
+                                            uint32_t (&plane)[K]) {
+  plane[K - 1] = S;
+  if (K >= 2) plane[0] = ~(S ^ M0);
+  if (K >= 3) plane[1] = ~(S ^ M1);
+  if (K >= 4) plane[2] = ~(S ^ M2);
+}
+
+// Q_MSE quantization of 32 coordinates u[0..32) (coordinate 32c + i in u[i])
+// against the positive thresholds t (boundaries times ||u||), bit planes
+// shifted into words (bit i = coordinate 32c + i).  K <= 3: every threshold
+// gives one thermometer plane T_j = [|u| > t_j]; the magnitude index
+// mu = T_0 + T_1 + T_2 has bits M1 = T_1 and M0 = T_0 ^ T_1 ^ T_2.  Each bit
+// costs one subtraction and one funnel shift.  K = 4: binary search of |u|
+// with integer masks.
+template <int K>
+__device__ __forceinline__ void quant32_mse(const uint32_t (&ur)[32], const float (&t)[8],
+                                            uint32_t (&plane)[K]) {
   uint32_t S = 0, M0 = 0, M1 = 0, M2 = 0;
+  if (K <= 3) {
+    uint32_t T0 = 0, T1 = 0, T2 = 0;
 #pragma unroll
-  for (int i = 31; i >= 0; --i) {
-    const float y = u[i];
-    const float a = fabsf(y);
-    const uint32_t s = gt_mask(y, 0.0f);
-    S = S + S - s;
-    float cm = c[0];
-    if (K == 2) {
-      const uint32_t m0 = gt_mask(a, t[0]);
-      M0 = M0 + M0 - m0;
-      if (RESID) cm = sel_mask(m0, c[1], c[0]);
-    } else if (K == 3) {
-      const uint32_t m1 = gt_mask(a, t[1]);
-      const uint32_t m0 = gt_mask(a, sel_mask(m1, t[2], t[0]));
-      M1 = M1 + M1 - m1;
-      M0 = M0 + M0 - m0;
-      if (RESID) cm = sel_mask(m1, sel_mask(m0, c[3], c[2]), sel_mask(m0, c[1], c[0]));
-    } else if (K == 4) {
+    for (int i = 31; i >= 0; --i) {
+      const float u = __uint_as_float(ur[i]);
+      const float a = fabsf(u);
+      S = shift_in(S, sub_bits(0.0f, u));
+      if (K >= 2) T0 = shift_in(T0, sub_bits(t[0], a));
+      if (K >= 3) {
+        T1 = shift_in(T1, sub_bits(t[1], a));
+        T2 = shift_in(T2, sub_bits(t[2], a));
+      }
+    }
+    M0 = K == 3 ? (T0 ^ T1 ^ T2) : T0;
+    M1 = T1;
+  } else {
+#pragma unroll
+    for (int i = 31; i >= 0; --i) {
+      const float u = __uint_as_float(ur[i]);
+      const float a = fabsf(u);
+      S = shift_in(S, sub_bits(0.0f, u));
       const uint32_t m2 = gt_mask(a, t[3]);
       const uint32_t m1 = gt_mask(a, sel_mask(m2, t[5], t[1]));
       const float tA = sel_mask(m2, t[6], t[2]), tB = sel_mask(m2, t[4], t[0]);
@@ -225,18 +263,46 @@ __device__ __forceinline__ void quant32(float (&u)[32], const float (&t)[8], con
       M1 = M1 + M1 - m1;
       M0 = M0 + M0 - m0;
     }
-    if (RESID) {
-      // u * inv - C[idx], C[idx] = +cm for u > 0 and -cm otherwise
-      const float negc = __uint_as_float(__float_as_uint(cm) ^ (s & 0x80000000u));
-      const float r = fmaf(y, inv, negc);
-      u[i] = r;
-      rr = fmaf(r, r, rr);
-    }
   }
-  plane[K - 1] = S;
-  if (K >= 2) plane[0] = ~(S ^ M0);
-  if (K >= 3) plane[1] = ~(S ^ M1);
-  if (K >= 4) plane[2] = ~(S ^ M2);
+  planes_from<K>(S, M0, M1, M2, plane);
+}
+
+// Q_prod's MSE stage (K <= 3 bits) for 32 coordinates, in the scaled unit
+// domain a' = |u| * inv with inv = 2^10 / ||u||: thresholds T_j = 2^10 t_j and
+// magnitudes C_j = 2^10 c_j (tc[j] = T_j - C_0, dc[j] = C_(j+1) - C_j).  With
+// e0 = a' - C_0 and d_j = T_j - a', the thermometer bit is sign(d_j), the step
+// [d_j < 0] is exact in {0, 1}, and e = e0 - sum_j step_j dc_j = a' - C_mu.
+// u[i] is replaced by 2^10 r = sign * e with the sign of the coordinate
+// (r = y - C[idx]); rr accumulates (2^10 r)^2.
+template <int K>
+__device__ __forceinline__ void quant32_prod(float (&v)[32], const float (&tc)[4], const float (&dc)[4],
+                                             float c0, float inv, uint32_t (&plane)[K], float& rr) {
+  uint32_t S = 0, T0 = 0, T1 = 0, T2 = 0;
+#pragma unroll
+  for (int i = 31; i >= 0; --i) {
+    const float u = v[i];
+    const uint32_t ds = sub_bits(0.0f, u);
+    S = shift_in(S, ds);
+    float e = fmaf(fabsf(u), inv, -c0);
+    if (K >= 2) {
+      const float e0 = e;
+      const float d0 = tc[0] - e0;
+      T0 = shift_in(T0, __float_as_uint(d0));
+      e = fmaf(step_neg(d0), -dc[0], e);
+      if (K >= 3) {
+        const float d1 = tc[1] - e0, d2 = tc[2] - e0;
+        T1 = shift_in(T1, __float_as_uint(d1));
+        T2 = shift_in(T2, __float_as_uint(d2));
+        e = fmaf(step_neg(d1), -dc[1], e);
+        e = fmaf(step_neg(d2), -dc[2], e);
+      }
+    }
+    rr = fmaf(e, e, rr);
+    // negative unless u > 0 (sign bit of 0 - u set)
+    v[i] = __uint_as_float(__float_as_uint(e) ^ (~ds & 0x80000000u));
+  }
+  const uint32_t M0 = K == 3 ? (T0 ^ T1 ^ T2) : T0;
+  planes_from<K>(S, M0, T1, 0u, plane);
 }
 
 // 32x32 bit transpose across the warp: lane t holds row t (bit i); returns
@@ -431,11 +497,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t ubase = tmem + (uint32_t)grp * buf_cols + lane_off;
     const TransposeCtl tctl = make_transpose_ctl(lane);
     const int half_levels = 1 << (K - 1);
-    float bpos[8], c1024[8];
+    float bpos[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      bpos[i] = i < half_levels - 1 ? qp.boundaries[half_levels + i] : 0.f;
-      c1024[i] = i < half_levels ? 1024.0f * qp.centroids[half_levels + i] : 0.f;
+    for (int i = 0; i < 8; ++i) bpos[i] = i < half_levels - 1 ? qp.boundaries[half_levels + i] : 0.f;
+    // Q_prod constants in the 2^10-scaled unit domain (see quant32_prod)
+    float tc[4], dc[4], c0s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tc[j] = dc[j] = 0.f;
+    if (PROD) {
+      c0s = 1024.0f * qp.centroids[half_levels];
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        if (j < half_levels - 1) {
+          tc[j] = 1024.0f * qp.boundaries[half_levels + j] - c0s;
+          dc[j] = 1024.0f * (qp.centroids[half_levels + j + 1] - qp.centroids[half_levels + j]);
+        }
+      }
     }
     for (int L = grp;; L += 2) {
       const int64_t tile = blockIdx.x + (int64_t)L * G;
@@ -458,27 +535,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         blk = a.codes + (seg0 * (a.seg_cap / 32) + (row0 - seg0 * a.seg_len) / 32) * (int64_t)(K * kDP);
       }
 
-      // pass 1: ||u|| over column chunks {0, 1} then {2, 3} (32 columns each);
-      // chunks 2 and 3 stay in registers for pass 2
-      uint32_t ur[2][32];
+      // pass 1: ||u|| over the four 32-column chunks; chunks 2 and 3 stay in
+      // registers for pass 2
+      uint32_t ra[32], rb[32];
       float ss0 = 0.f, ss1 = 0.f, ss2 = 0.f, ss3 = 0.f;
+      auto sumsq = [&](const uint32_t (&r)[32]) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        tmem_ld32(ubase + (uint32_t)(64 * h), ur[0]);
-        tmem_ld32(ubase + (uint32_t)(64 * h + 32), ur[1]);
-        tmem_ld_wait<2>(ur);
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float v0 = __uint_as_float(ur[c][i]), v1 = __uint_as_float(ur[c][i + 1]);
-            const float v2 = __uint_as_float(ur[c][i + 2]), v3 = __uint_as_float(ur[c][i + 3]);
-            ss0 = fmaf(v0, v0, ss0);
-            ss1 = fmaf(v1, v1, ss1);
-            ss2 = fmaf(v2, v2, ss2);
-            ss3 = fmaf(v3, v3, ss3);
-          }
-      }
+        for (int i = 0; i < 32; i += 4) {
+          const float v0 = __uint_as_float(r[i]), v1 = __uint_as_float(r[i + 1]);
+          const float v2 = __uint_as_float(r[i + 2]), v3 = __uint_as_float(r[i + 3]);
+          ss0 = fmaf(v0, v0, ss0);
+          ss1 = fmaf(v1, v1, ss1);
+          ss2 = fmaf(v2, v2, ss2);
+          ss3 = fmaf(v3, v3, ss3);
+        }
+      };
+      tmem_ld32(ubase, ra);
+      tmem_ld32(ubase + 32u, rb);
+      tmem_ld_wait2(ra, rb);
+      sumsq(ra);
+      sumsq(rb);
+      tmem_ld32(ubase + 64u, ra);
+      tmem_ld32(ubase + 96u, rb);
+      tmem_ld_wait2(ra, rb);
+      sumsq(ra);
+      sumsq(rb);
       const float nu = sqrtf((ss0 + ss1) + (ss2 + ss3));  // ||u|| = sqrt(d_pad) ||x||
       if (valid) a.norms[slot] = nu * qp.inv_sqrt_dpad;
       float th[8];
@@ -487,58 +568,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = nu > 0.f ? 1024.0f / nu : 0.f;
       float rr = 0.f;
       uint32_t rowq[K][4];
-      // pass 2: chunks 2 and 3 from registers, then chunks 0 and 1 again
-#pragma unroll
-      for (int h = 1; h >= 0; --h) {
-        if (h == 0) {
-          tmem_ld32(ubase, ur[0]);
-          tmem_ld32(ubase + 32u, ur[1]);
-          tmem_ld_wait<2>(ur);
-          if (!PROD) {
-            // u has been read: the buffer is free for the next tile
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bar_acce[grp]));
-          }
-        }
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = 2 * h + cc;
+
+      // quantize chunk c (coordinates 32c .. 32c+31) held in r
+      auto process = [&](const int c, const uint32_t (&r)[32]) {
+        uint32_t planes[K];
+        if (PROD) {
           float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ur[cc][i]);
-          uint32_t planes[K];
-          quant32<K, PROD>(v, th, c1024, inv, planes, rr);
-          if (MODE == MODE_MSE_BLOCK) {
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          quant32_prod<(PROD ? K : 1)>(v, tc, dc, c0s, inv, *reinterpret_cast<uint32_t(*)[(PROD ? K : 1)]>(planes), rr);
+          // 2^10 r as fp16 hi (columns 32c .. 32c+15) and lo (32c+16 .. 32c+31)
+          // parts.  |r| <= 2, so 2^10 r is far below the fp16 maximum; hi keeps
+          // the top 11 significant bits (exact in fp16), lo = 2^10 r - hi is
+          // rounded to fp16, about 22 bits in all.  The sign of S r does not
+          // change with the scale.
 #pragma unroll
-            for (int p = 0; p < K; ++p) {
-              const uint32_t word = transpose32(valid ? planes[p] : 0u, tctl);
-              if (have) blk[p * kDP + 32 * c + lane] = word;
-            }
-          } else {
+          for (int g = 0; g < 2; ++g) {  // coordinates 32c + 16g .. +15
+            uint32_t hiw[8], low[8];
 #pragma unroll
-            for (int p = 0; p < K; ++p) rowq[p][c] = planes[p];
-          }
-          if (PROD) {
-            // this chunk's residual as fp16 hi (columns 32c .. 32c+15) and lo
-            // (32c+16 .. 32c+31) parts: |r| <= 2 so 2^10 r stays below the fp16
-            // maximum and its lo part out of the subnormal range; the sign of S r
-            // is unchanged by the scale.
-            uint32_t hiw[16], low[16];
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-              const float r0 = v[2 * q], r1 = v[2 * q + 1];
-              const __half2 hv = __floats2half2_rn(r0, r1);
-              const float2 hf = __half22float2(hv);
-              const __half2 l = __floats2half2_rn(r0 - hf.x, r1 - hf.y);
+            for (int q = 0; q < 8; ++q) {
+              const float r0 = v[16 * g + 2 * q], r1 = v[16 * g + 2 * q + 1];
+              const float h0 = __uint_as_float(__float_as_uint(r0) & 0xFFFFE000u);
+              const float h1 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
+              const __half2 hv = __floats2half2_rn(h0, h1);
+              const __half2 lv = __floats2half2_rn(r0 - h0, r1 - h1);
               hiw[q] = *reinterpret_cast<const uint32_t*>(&hv);
-              low[q] = *reinterpret_cast<const uint32_t*>(&l);
+              low[q] = *reinterpret_cast<const uint32_t*>(&lv);
             }
-            tmem_st16(ubase + (uint32_t)(32 * c), hiw);
-            tmem_st16(ubase + (uint32_t)(32 * c + 16), low);
+            tmem_st8(ubase + (uint32_t)(32 * c + 8 * g), hiw);
+            tmem_st8(ubase + (uint32_t)(32 * c + 16 + 8 * g), low);
           }
+        } else {
+          quant32_mse<K>(r, th, planes);
         }
+        if (MODE == MODE_MSE_BLOCK) {
+#pragma unroll
+          for (int p = 0; p < K; ++p) {
+            const uint32_t word = transpose32(valid ? planes[p] : 0u, tctl);
+            if (have) blk[p * kDP + 32 * c + lane] = word;
+          }
+        } else {
+#pragma unroll
+          for (int p = 0; p < K; ++p) rowq[p][c] = planes[p];
+        }
+      };
+
+      // pass 2: each chunk's reload from TMEM overlaps the previous chunk's work
+      process(2, ra);
+      tmem_ld32(ubase, ra);
+      process(3, rb);
+      tmem_ld_wait1(ra);
+      tmem_ld32(ubase + 32u, rb);
+      process(0, ra);
+      tmem_ld_wait1(rb);
+      if (!PROD) {
+        // u has been read: the buffer is free for the next tile
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar_acce[grp]));
       }
+      process(1, rb);
       if (MODE != MODE_MSE_BLOCK && valid) {
         uint4* dst = reinterpret_cast<uint4*>(a.codes + slot * (int64_t)(K * 4));
 #pragma unroll
@@ -557,12 +646,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           if (32 * c < m) {
-            uint32_t z[1][32];
-            tmem_ld32(zbase + (uint32_t)(32 * c), z[0]);
-            tmem_ld_wait<1>(z);
+            uint32_t z[32];
+            tmem_ld32(zbase + (uint32_t)(32 * c), z);
+            tmem_ld_wait1(z);
             uint32_t neg = 0;
 #pragma unroll
-            for (int i = 31; i >= 0; --i) neg = (neg << 1) | (z[0][i] >> 31);
+            for (int i = 31; i >= 0; --i) neg = shift_in(neg, z[i]);
             sw[c] = ~neg;  // bit i = [ (S r)_(32c+i) >= 0 ]
           } else {
             sw[c] = 0u;
