@@ -9,11 +9,18 @@ namespace {
 template <int K, int MODE>
 cudaError_t launch_one(const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,
                        cudaStream_t st) {
-  auto kern = encode_tc_kernel<__nv_bfloat16, K, MODE>;
   const int smem = (int)smem_bytes(MODE, qp.m);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  kern<<<ctas, kThreads, smem, st>>>(map, qp, a);
+  if constexpr (MODE == MODE_PROD) {
+    auto kern = encode_prod_kernel<__nv_bfloat16, K>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, kThreadsP, smem, st>>>(map, qp, a);
+  } else {
+    auto kern = encode_tc_kernel<__nv_bfloat16, K, MODE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, kThreads, smem, st>>>(map, qp, a);
+  }
   return cudaGetLastError();
 }
 
