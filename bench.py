@@ -20,7 +20,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -78,56 +77,61 @@ def workload_bytes(cfg, k_words, k_signs, v_words):
 
 
 class ClockSampler:
-    """nvidia-smi samples during the timed region (median SM MHz, throttle reasons)."""
+    """SM clock and clock-event reasons sampled through NVML every few ms
+    during the timed region (read-only queries); falls back to nvidia-smi.
+    Reports the median SM MHz under load, the maximum SM MHz and every
+    slowdown reason seen active."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, index):
+    def __init__(self, index, period_s=0.005):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.period = period_s
+        self.sm, self.reasons = [], set()
+        self.smax = None
+        self.stop_evt = threading.Event()
+        self.t = None
+        self.err = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except Exception:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            masks = [(nm, getattr(pynvml, attr)) for nm, attr in self.REASONS]
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            def loop():
+                while True:
+                    try:
+                        self.sm.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                        r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        for nm, mk in masks:
+                            if r & mk:
+                                self.reasons.add(nm)
+                    except Exception as e:  # keep the samples taken so far
+                        self.err = str(e)
+                        return
+                    if self.stop_evt.wait(self.period):
+                        return
+
+            self.t = threading.Thread(target=loop, daemon=True)
+            self.t.start()
+        except Exception as e:
+            self.err = f"nvml unavailable: {e}"
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.t is not None:
+            self.stop_evt.set()
+            self.t.join(timeout=5)
+        out = {"sm_mhz": statistics.median(self.sm) if self.sm else None,
+               "sm_max_mhz": self.smax, "reasons": sorted(self.reasons), "samples": len(self.sm)}
+        if self.err and not self.sm:
+            out["reasons"] = [self.err]
+        return out
 
 
 class OracleSample:
@@ -269,7 +273,11 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks = ClockSampler(local)
+    try:
+        nvml_index = torch.cuda._get_nvml_device_index(local)  # honours CUDA_VISIBLE_DEVICES
+    except Exception:
+        nvml_index = local
+    clocks = ClockSampler(nvml_index)
     clocks.start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)

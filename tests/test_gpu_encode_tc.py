@@ -81,16 +81,17 @@ def test_tc_encode_prod(d, m, bits, dtype, n):
     assert_close_rel(rnorms.cpu().numpy(), e["rnorms"], 1e-30, what="rnorms", mask=~bad)
 
 
-@pytest.mark.parametrize("layout", [tq.LAYOUT_ROW, tq.LAYOUT_BLOCK32])
-def test_tc_encode_segments_with_capacity(layout):
-    # 5 segments of 96 vectors into slots of 160: slots >= 96 untouched
+@pytest.mark.parametrize("layout,seg,cap,ns", [(tq.LAYOUT_ROW, 96, 160, 5),
+                                               (tq.LAYOUT_BLOCK32, 96, 160, 5),
+                                               (tq.LAYOUT_ROW, 1184, 1216, 9),
+                                               (tq.LAYOUT_BLOCK32, 32, 64, 70)])
+def test_tc_encode_segments_with_capacity(layout, seg, cap, ns):
+    # ns segments of seg vectors into slots of cap: slots >= seg untouched
     ora, lib = make_pair(128, 3, False, seed=5)
-    seg, cap, ns = 96, 160, 5
     x = synth.gaussian_vectors(seg * ns, 128, seed=11, dtype="float16", device=DEV)
     codes, norms = tq.tq_encode_mse(lib, x, layout=layout, seg_len=seg, seg_cap=cap)
     torch.cuda.synchronize()
     w = u32(codes)
-    words = 3 * 128 // 32
     for s in range(ns):
         e = ora.encode(x_np(x[seg * s:seg * (s + 1)]), layout="row")
         if layout == tq.LAYOUT_ROW:
@@ -103,7 +104,26 @@ def test_tc_encode_segments_with_capacity(layout):
         check_codes(gi, e["idx"], e["y"], ora.boundaries, 128)
         assert_close_rel(norms[cap * s:cap * s + seg].cpu().numpy(), e["norms"], 1e-30)
         assert np.all(norms[cap * s + seg:cap * (s + 1)].cpu().numpy() == 0)
-    assert words == 12
+
+
+def test_tc_encode_prod_segments():
+    # Q_prod rows land in slot s * cap + pos of their segment
+    ora, lib = make_pair(128, 3, True, seed=6)
+    seg, cap, ns = 160, 192, 7
+    x = synth.gaussian_vectors(seg * ns, 128, seed=13, dtype="bfloat16", device=DEV)
+    codes, signs, norms, rnorms = tq.tq_encode_prod(lib, x, seg_len=seg, seg_cap=cap)
+    torch.cuda.synchronize()
+    w, sg = u32(codes), u32(signs)
+    for s in range(ns):
+        e = ora.encode(x_np(x[seg * s:seg * (s + 1)]))
+        gi = o.unpack_row(w[cap * s:cap * s + seg], ora.k, 128)
+        _, bad = check_codes(gi, e["idx"], e["y"], ora.boundaries, 128)
+        nsg = check_signs(sg[cap * s:cap * s + seg], e["signs"], e["z"], e["rho64"], ora.m, skip_rows=bad)
+        assert nsg <= 1e-4 * seg * ora.m
+        assert_close_rel(norms[cap * s:cap * s + seg].cpu().numpy(), e["norms"], 1e-30)
+        assert_close_rel(rnorms[cap * s:cap * s + seg].cpu().numpy(), e["rnorms"], 1e-30, mask=~bad)
+        assert np.all(w[cap * s + seg:cap * (s + 1)] == 0)
+        assert np.all(sg[cap * s + seg:cap * (s + 1)] == 0)
 
 
 def test_tc_encode_many_tiles_per_cta():

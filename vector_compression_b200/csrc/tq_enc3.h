@@ -23,8 +23,31 @@ constexpr uint32_t kRotBytes = kDP * kDP * 2;      // 32 KB rotation operand
 
 enum { MODE_MSE_ROW = 0, MODE_MSE_BLOCK = 1, MODE_PROD = 2 };
 
+// Division by a fixed d (1 <= d < 2^31) of n < 2^31 as a multiply and shift:
+// with s = ceil(log2 d) and M = floor(2^(32+s) / d) + 1 = 2^32 + mul, the
+// product n M / 2^(32+s) exceeds n / d by less than n / 2^(32+s) < 1 / (2d),
+// too little to reach the next integer, so
+// floor(n / d) = (umulhi(n, mul) + n) >> s  (the sum stays below 2^32).
+struct FastDiv {
+  uint32_t d, mul, shift;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.shift = 0;
+  while (((uint64_t)1 << f.shift) < d) ++f.shift;
+  f.mul = (uint32_t)((((uint64_t)1 << (32 + f.shift)) / d) - ((uint64_t)1 << 32) + 1);
+  return f;
+}
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.mul) + n) >> f.shift;
+}
+#endif
+
 struct Args {
   int64_t n_vec, seg_len, seg_cap, n_tiles;
+  FastDiv seg_div;  // division by seg_len
   uint32_t* codes;
   uint32_t* signs;
   float* norms;

@@ -35,7 +35,7 @@ bool try_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_v
   if ((qp.d * 2) % 16 != 0 || (ld * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(x) & 15u) != 0)
     return false;
   if (seg_len <= 0 || seg_len % 32 != 0 || n_vec % seg_len != 0) return false;
-  if (n_vec > ((int64_t)1 << 31) - 2 * kRows) return false;
+  if (n_vec > ((int64_t)1 << 31) - 2 * kRows) return false;  // rows (and tile rows) < 2^31
   if (qp.k < 1 || qp.k > (prod ? 3 : 4)) return false;
   if (prod && qp.m != 64 && qp.m != 128) return false;
   if (!err_word) return false;
@@ -61,6 +61,7 @@ bool try_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_v
   a.n_vec = n_vec;
   a.seg_len = seg_len;
   a.seg_cap = seg_cap;
+  a.seg_div = make_fastdiv((uint32_t)seg_len);
   a.n_tiles = (n_vec + kRows - 1) / kRows;
   a.codes = codes;
   a.signs = signs;

@@ -61,24 +61,31 @@ __device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
                : "memory");
 }
 
+// One test of the phase with the given parity; the thread may be suspended
+// (up to the hint, in ns) until the phase completes.
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(20000u)
+      : "memory");
+  return done != 0;
+}
+
 // Bounded wait for the phase with the given parity: false (and the device
 // error word set) if it has not completed within ~2^31 cycles.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
+  if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
-  while (true) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (done) return true;
+  while (!mbar_try(bar, parity)) {
     if (clock64() - t0 > (1LL << 31)) {
       atomicCAS(err, 0u, (unsigned)TQ_ERR_TIMEOUT);
       return false;
     }
   }
+  return true;
 }
 
 // Warp-uniform form: every lane waits, the warp proceeds only if all saw it.
@@ -555,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t row = tile * kRows + quarter * 32 + lane;
       const bool valid = row < a.n_vec;
       const bool have = tile * kRows + quarter * 32 < a.n_vec;  // any valid row in this warp
-      const int64_t seg = valid ? row / a.seg_len : 0;
+      const int64_t seg = valid ? (int64_t)fastdiv((uint32_t)row, a.seg_div) : 0;
       const int64_t pos = valid ? row - seg * a.seg_len : 0;
       const int64_t slot = seg * a.seg_cap + pos;
       // BLOCK32: the warp's 32 rows are one block of one segment (segments hold
@@ -563,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t* blk = nullptr;
       if (MODE == MODE_MSE_BLOCK) {
         const int64_t row0 = tile * kRows + quarter * 32;
-        const int64_t seg0 = row0 / a.seg_len;
+        const int64_t seg0 = (int64_t)fastdiv((uint32_t)row0, a.seg_div);
         blk = a.codes + (seg0 * (a.seg_cap / 32) + (row0 - seg0 * a.seg_len) / 32) * (int64_t)(K * kDP);
       }
 
@@ -950,7 +957,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
       if (lane == 0) mbar_arrive(smem_u32(&bar_normx));
       const int64_t row = tile * kRows + rloc;
       const bool valid = row < a.n_vec;
-      const int64_t seg = valid ? row / a.seg_len : 0;
+      const int64_t seg = valid ? (int64_t)fastdiv((uint32_t)row, a.seg_div) : 0;
       const int64_t slot = seg * a.seg_cap + (valid ? row - seg * a.seg_len : 0);
       if (!mbar_wait_warp(smem_u32(&bar_normx), (uint32_t)L & 1u, a.err)) { ok = false; break; }
       const float4 q = *reinterpret_cast<const float4*>(&ss_part[b][rloc][0]);
