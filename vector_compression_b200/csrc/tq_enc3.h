@@ -61,6 +61,10 @@ inline uint32_t smem_bytes(int mode, int m) {
   return kRotBytes + (mode == MODE_PROD ? (uint32_t)m * kDP * 2 : 0u) + kStages * kTileBytes + 1024;
 }
 
+// Threads per vector of the Q_prod encoder (2, or 4 with TQ_PROD_TPR=4 in
+// the environment).
+int prod_tpr();
+
 cudaError_t launch_f16(int mode, const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,
                        cudaStream_t st);
 cudaError_t launch_bf16(int mode, const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,

@@ -14,15 +14,17 @@
 //   warp 0      TMA producer: tiles of 128 consecutive input rows, two
 //               128-byte-swizzled boxes of 64 columns each, into a 4-stage ring;
 //   warp 1      TMEM allocator and MMA issuer (one elected thread);
-//   warps 2..9  two epilogue groups of four warps; group g owns TMEM buffer g
-//               and every second tile.  Thread (warp w, lane l) reads TMEM lane
-//               32 (w % 4) + l, i.e. one vector: its 128 values of u, the norm
-//               n = ||u|| / sqrt(d_pad), the sign plane and the binary search of
-//               |u| against the positive boundaries scaled by ||u||.
-// Q_prod: the epilogue writes r = u / ||u|| - C[idx] (times 2^10, split into fp16
-// hi + lo parts) back into its TMEM lane, a second MMA forms S r for the tile
-// (A = r from TMEM, B = S from shared memory) and the epilogue reads its row to
-// form the QJL sign words.
+//   the rest    the epilogue, reading u from TMEM (warp w may read TMEM lanes
+//               32 (w % 4) .. +31, i.e. those vectors of the tile).
+// Q_MSE (encode_tc_kernel): two epilogue groups of four warps, group g owns
+// TMEM buffer g and every second tile; one thread per vector computes
+// n = ||u|| / sqrt(d_pad) and the bit planes (sign plane and thermometer
+// planes of |u| against the positive boundaries scaled by ||u||).
+// Q_prod (encode_prod_kernel): one group of 16 warps, four threads per vector
+// (32 columns each); the epilogue writes r = u / ||u|| - C[idx] (times 2^10,
+// split into fp16 hi + lo parts) back over u, a second MMA forms S r (A = r
+// from TMEM, B = S from shared memory) while the next tile is quantized, and
+// the epilogue then reads its rows of S r for the QJL sign words.
 // Exact boundary ties on the negative side resolve toward zero here (the
 // oracle resolves them to the lower cell); such values lie inside the parity
 // window by definition.
@@ -279,41 +281,9 @@ __device__ __forceinline__ void quant32_mse(const uint32_t (&ur)[32], const floa
 // magnitudes C_j = 2^10 c_j (tc[j] = T_j - C_0, dc[j] = C_(j+1) - C_j).  With
 // e0 = a' - C_0 and d_j = T_j - a', the thermometer bit is sign(d_j), the step
 // [d_j < 0] is exact in {0, 1}, and e = e0 - sum_j step_j dc_j = a' - C_mu.
-// u[i] is replaced by 2^10 r = sign * e with the sign of the coordinate
-// (r = y - C[idx]); rr accumulates (2^10 r)^2.
-template <int K>
-__device__ __forceinline__ void quant32_prod(float (&v)[32], const float (&tc)[4], const float (&dc)[4],
-                                             float c0, float inv, uint32_t (&plane)[K], float& rr) {
-  uint32_t S = 0, T0 = 0, T1 = 0, T2 = 0;
-#pragma unroll
-  for (int i = 31; i >= 0; --i) {
-    const float u = v[i];
-    const uint32_t ds = sub_bits(0.0f, u);
-    S = shift_in(S, ds);
-    float e = fmaf(fabsf(u), inv, -c0);
-    if (K >= 2) {
-      const float e0 = e;
-      const float d0 = tc[0] - e0;
-      T0 = shift_in(T0, __float_as_uint(d0));
-      e = fmaf(step_neg(d0), -dc[0], e);
-      if (K >= 3) {
-        const float d1 = tc[1] - e0, d2 = tc[2] - e0;
-        T1 = shift_in(T1, __float_as_uint(d1));
-        T2 = shift_in(T2, __float_as_uint(d2));
-        e = fmaf(step_neg(d1), -dc[1], e);
-        e = fmaf(step_neg(d2), -dc[2], e);
-      }
-    }
-    rr = fmaf(e, e, rr);
-    // negative unless u > 0 (sign bit of 0 - u set)
-    v[i] = __uint_as_float(__float_as_uint(e) ^ (~ds & 0x80000000u));
-  }
-  const uint32_t M0 = K == 3 ? (T0 ^ T1 ^ T2) : T0;
-  planes_from<K>(S, M0, T1, 0u, plane);
-}
-
-// Q_prod's MSE stage as in quant32_prod, with the sign plane taken from the
-// sign bits of u: NS (bit set = negative) is shifted in and S = ~NS per word.
+// v[i] becomes 2^10 r = +-e with the sign of the coordinate (r = y - C[idx]);
+// rr accumulates (2^10 r)^2.  The sign plane comes from the sign bits of u:
+// NS (bit set = negative) is shifted in and S = ~NS per word.
 // An exactly zero coordinate of a nonzero vector then takes the upper middle
 // cell (a tie at the middle boundary, y = 0 = B); the caller forces S = 0 for
 // zero vectors.  The residual keeps the coordinate's sign bit.
@@ -382,22 +352,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, QParams qp, Args a) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages];
-  __shared__ __align__(8) uint64_t bar_accf[2], bar_acce[2], bar_aready[2], bar_zf[2], bar_done;
+  __shared__ __align__(8) uint64_t bar_accf[2], bar_acce[2], bar_done;
   __shared__ uint32_t tmem_base_s;
-  constexpr bool PROD = MODE == MODE_PROD;
   constexpr bool BF16 = sizeof(T) == 2 && !std::is_same<T, __half>::value;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m = qp.m;
   // 1024-byte alignment for the swizzled tiles
   unsigned char* smem =
       smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   unsigned char* rot = smem;
-  unsigned char* smat = smem + kRotBytes;
-  unsigned char* stages = smat + (PROD ? m * kDP * 2 : 0);
-  const uint32_t tmem_cols = PROD ? 512u : 256u;
-  const uint32_t buf_cols = PROD ? 256u : 128u;
+  unsigned char* stages = smem + kRotBytes;
+  constexpr uint32_t tmem_cols = 256u;
+  constexpr uint32_t buf_cols = 128u;
 
-  // ---- setup: rotation operand B[n][k] = H[n][k] D_k (+-1) and S, barriers, TMEM
+  // ---- setup: rotation operand B[n][k] = H[n][k] D_k (+-1), barriers, TMEM
   {
     const uint16_t one = BF16 ? 0x3F80u : 0x3C00u;
     for (int e = tid; e < kDP * (kDP / 8); e += kThreads) {
@@ -416,13 +383,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       w.w = v[6] | ((uint32_t)v[7] << 16);
       *reinterpret_cast<uint4*>(rot + core_offset(n, kc * 8, kDP)) = w;
     }
-    if (PROD) {
-      for (int e = tid; e < m * (kDP / 8); e += kThreads) {
-        const int row = e / (kDP / 8), kc = e % (kDP / 8);
-        const uint4 w = *reinterpret_cast<const uint4*>(qp.S16 + (size_t)row * kDP + kc * 8);
-        *reinterpret_cast<uint4*>(smat + core_offset(row, kc * 8, m)) = w;
-      }
-    }
   }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -432,8 +392,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&bar_accf[b]), 1);
       mbar_init(smem_u32(&bar_acce[b]), 4);
-      mbar_init(smem_u32(&bar_aready[b]), 4);
-      mbar_init(smem_u32(&bar_zf[b]), 1);
     }
     mbar_init(smem_u32(&bar_done), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -476,20 +434,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t fmt = BF16 ? 1u : 0u;
       const uint32_t idesc1 = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kDP >> 3) << 17) |
                               ((uint32_t)(kRows >> 4) << 24);
-      const uint32_t idesc2 =
-          (1u << 4) | ((uint32_t)(m >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
       const uint32_t rot_base = smem_u32(rot);
-      const uint32_t s_base = smem_u32(smat);
-      const uint32_t s_lbo = (uint32_t)(m / 8) * 128u;
-      bool ok = true;
-      int L = 0;
-      for (;; ++L) {
+      for (int L = 0;; ++L) {
         const int64_t tile = blockIdx.x + (int64_t)L * G;
         const bool have = tile < a.n_tiles;
         if (have) {
           const int s = L % kStages, b = L & 1;
-          if (!mbar_wait(smem_u32(&bar_full[s]), (L / kStages) & 1, a.err)) { ok = false; break; }
-          if (L >= 2 && !mbar_wait(smem_u32(&bar_acce[b]), ((L >> 1) - 1) & 1, a.err)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&bar_full[s]), (L / kStages) & 1, a.err)) break;
+          if (L >= 2 && !mbar_wait(smem_u32(&bar_acce[b]), ((L >> 1) - 1) & 1, a.err)) break;
           tc_fence_after();
           const uint32_t a_base = smem_u32(stages + s * kTileBytes);
           const uint32_t d_tmem = tmem + (uint32_t)b * buf_cols;
@@ -502,30 +454,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(smem_u32(&bar_empty[s]));
           tc_commit(smem_u32(&bar_accf[b]));
         }
-        if (PROD && L >= 1) {
-          // S r for the previous tile, once its epilogue has written r
-          const int Lp = L - 1, b = Lp & 1;
-          if (!mbar_wait(smem_u32(&bar_aready[b]), (Lp >> 1) & 1, a.err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_tmem = tmem + (uint32_t)b * buf_cols;
-          const uint32_t z_tmem = a_tmem + 128u;
-#pragma unroll
-          for (int pass = 0; pass < 2; ++pass) {  // hi, then lo parts of r
-#pragma unroll
-            for (int t = 0; t < kDP / 16; ++t) {
-              const uint32_t acol = (uint32_t)(32 * (t >> 1) + 16 * pass + 8 * (t & 1));
-              const uint64_t bd = desc_noswz(s_base + (uint32_t)(2 * t) * s_lbo, s_lbo, 128u);
-              mma_ts(z_tmem, a_tmem + acol, bd, idesc2, (pass | t) ? 1u : 0u);
-            }
-          }
-          tc_commit(smem_u32(&bar_zf[b]));
-        }
         if (!have) break;
       }
       // every MMA issued above has completed before TMEM is released
       tc_commit(smem_u32(&bar_done));
       mbar_wait(smem_u32(&bar_done), 0, a.err);
-      (void)ok;
     }
   } else {
     // ---------------------------------------------------------------- epilogue
@@ -539,20 +472,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     float bpos[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) bpos[i] = i < half_levels - 1 ? qp.boundaries[half_levels + i] : 0.f;
-    // Q_prod constants in the 2^10-scaled unit domain (see quant32_prod)
-    float tc[4], dc[4], c0s = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) tc[j] = dc[j] = 0.f;
-    if (PROD) {
-      c0s = 1024.0f * qp.centroids[half_levels];
-#pragma unroll
-      for (int j = 0; j < 3; ++j) {
-        if (j < half_levels - 1) {
-          tc[j] = 1024.0f * qp.boundaries[half_levels + j] - c0s;
-          dc[j] = 1024.0f * (qp.centroids[half_levels + j + 1] - qp.centroids[half_levels + j]);
-        }
-      }
-    }
     for (int L = grp;; L += 2) {
       const int64_t tile = blockIdx.x + (int64_t)L * G;
       if (tile >= a.n_tiles) break;
@@ -599,47 +518,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait2(ra, rb);
       sumsq(ra);
       sumsq(rb);
-      const float nu = sqrtf((ss0 + ss1) + (ss2 + ss3));  // ||u|| = sqrt(d_pad) ||x||
+      const float ssum = (ss0 + ss1) + (ss2 + ss3);       // ||u||^2 = d_pad ||x||^2
+      const float nu = ssum > 0.f ? ssum * rsqrtf(ssum) : 0.f;
       if (valid) a.norms[slot] = nu * qp.inv_sqrt_dpad;
       float th[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) th[i] = bpos[i] * nu;
-      const float inv = nu > 0.f ? 1024.0f / nu : 0.f;
-      float rr = 0.f;
       uint32_t rowq[K][4];
 
       // quantize chunk c (coordinates 32c .. 32c+31) held in r
       auto process = [&](const int c, const uint32_t (&r)[32]) {
         uint32_t planes[K];
-        if (PROD) {
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          quant32_prod<(PROD ? K : 1)>(v, tc, dc, c0s, inv, *reinterpret_cast<uint32_t(*)[(PROD ? K : 1)]>(planes), rr);
-          // 2^10 r as fp16 hi (columns 32c .. 32c+15) and lo (32c+16 .. 32c+31)
-          // parts.  |r| <= 2, so 2^10 r is far below the fp16 maximum; hi keeps
-          // the top 11 significant bits (exact in fp16), lo = 2^10 r - hi is
-          // rounded to fp16, about 22 bits in all.  The sign of S r does not
-          // change with the scale.
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {  // coordinates 32c + 16g .. +15
-            uint32_t hiw[8], low[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float r0 = v[16 * g + 2 * q], r1 = v[16 * g + 2 * q + 1];
-              const float h0 = __uint_as_float(__float_as_uint(r0) & 0xFFFFE000u);
-              const float h1 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
-              const __half2 hv = __floats2half2_rn(h0, h1);
-              const __half2 lv = __floats2half2_rn(r0 - h0, r1 - h1);
-              hiw[q] = *reinterpret_cast<const uint32_t*>(&hv);
-              low[q] = *reinterpret_cast<const uint32_t*>(&lv);
-            }
-            tmem_st8(ubase + (uint32_t)(32 * c + 8 * g), hiw);
-            tmem_st8(ubase + (uint32_t)(32 * c + 16 + 8 * g), low);
-          }
-        } else {
-          quant32_mse<K>(r, th, planes);
-        }
+        quant32_mse<K>(r, th, planes);
         if (MODE == MODE_MSE_BLOCK) {
 #pragma unroll
           for (int p = 0; p < K; ++p) {
@@ -660,51 +550,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(ubase + 32u, rb);
       process(0, ra);
       tmem_ld_wait1(rb);
-      if (!PROD) {
-        // u has been read: the buffer is free for the next tile
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar_acce[grp]));
-      }
+      // u has been read: the buffer is free for the next tile
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar_acce[grp]));
       process(1, rb);
       if (MODE != MODE_MSE_BLOCK && valid) {
         uint4* dst = reinterpret_cast<uint4*>(a.codes + slot * (int64_t)(K * 4));
 #pragma unroll
         for (int p = 0; p < K; ++p) dst[p] = make_uint4(rowq[p][0], rowq[p][1], rowq[p][2], rowq[p][3]);
-      }
-      if (PROD) {
-        if (valid) a.rnorms[slot] = sqrtf(rr) * (1.0f / 1024.0f);
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar_aready[grp]));
-        if (!mbar_wait_warp(smem_u32(&bar_zf[grp]), par, a.err)) break;
-        tc_fence_after();
-        const uint32_t zbase = ubase + 128u;
-        uint32_t sw[8];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (32 * c < m) {
-            uint32_t z[32];
-            tmem_ld32(zbase + (uint32_t)(32 * c), z);
-            tmem_ld_wait1(z);
-            uint32_t neg = 0;
-#pragma unroll
-            for (int i = 31; i >= 0; --i) neg = shift_in(neg, z[i]);
-            sw[c] = ~neg;  // bit i = [ (S r)_(32c+i) >= 0 ]
-          } else {
-            sw[c] = 0u;
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bar_acce[grp]));
-        if (valid) {
-          if (m == 128)
-            *reinterpret_cast<uint4*>(a.signs + slot * 4) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-          else
-            *reinterpret_cast<uint2*>(a.signs + slot * 2) = make_uint2(sw[0], sw[1]);
-        }
       }
     }
   }
@@ -720,18 +574,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ Q_prod kernel
 
-// Q_prod: one epilogue group of 16 warps works on every tile; thread (warp w,
-// lane l) owns TMEM lane 32 (w % 4) + l (one vector) and the 32 columns
-// 32 c .. 32 c + 31, c = (w - 2) / 4.  TMEM holds two tiles, each with a
+// Q_prod: one epilogue group of 4 TPR warps works on every tile; thread
+// (warp w, lane l) owns TMEM lane 32 (w % 4) + l (one vector) and the
+// 128 / TPR columns of column group (w - 2) / 4.  TMEM holds two tiles, each with a
 // 128-column slot for u (rewritten in place with the fp16 hi/lo residual, the
 // A operand of S r) and a 128-column slot for z = S r.  The S r MMA of tile L
 // runs while the epilogue quantizes tile L + 1; the signs of tile L are read
 // after that, so no warp waits for an MMA in steady state.
-constexpr int kEpiWarpsP = 16;
-constexpr int kThreadsP = 64 + 32 * kEpiWarpsP;  // 576
+template <int TPR>
+constexpr int prod_threads() { return 64 + 32 * 4 * TPR; }
 
-template <typename T, int K>
-__global__ void __launch_bounds__(kThreadsP, 1)
+template <typename T, int K, int TPR>
+__global__ void __launch_bounds__(prod_threads<TPR>(), 1)
     encode_prod_kernel(const __grid_constant__ CUtensorMap xmap, QParams qp, Args a) {
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages];
@@ -740,6 +594,10 @@ __global__ void __launch_bounds__(kThreadsP, 1)
   __shared__ __align__(16) float rr_part[2][kRows][4];  // partial ||2^10 r||^2
   __shared__ uint32_t tmem_base_s;
   constexpr bool BF16 = !std::is_same<T, __half>::value;
+  constexpr int kEpiWarpsP = 4 * TPR;            // epilogue warps
+  constexpr int kThreadsP = prod_threads<TPR>();
+  constexpr int CPT = 4 / TPR;                   // 32-column chunks per thread
+  static_assert(TPR == 2 || TPR == 4, "two or four threads per vector");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m = qp.m;
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -779,11 +637,11 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&bar_accf[b]), 1);
-      mbar_init(smem_u32(&bar_aready[b]), kEpiWarpsP);
+      mbar_init(smem_u32(&bar_aready[b]), 32 * kEpiWarpsP);  // every epilogue thread arrives
       mbar_init(smem_u32(&bar_zf[b]), 1);
-      mbar_init(smem_u32(&bar_zempty[b]), kEpiWarpsP);
+      mbar_init(smem_u32(&bar_zempty[b]), 32 * kEpiWarpsP);
     }
-    mbar_init(smem_u32(&bar_normx), kEpiWarpsP);
+    mbar_init(smem_u32(&bar_normx), 32 * kEpiWarpsP);
     mbar_init(smem_u32(&bar_done), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -877,7 +735,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int ew = warp - 2;        // 0..15
-    const int c = ew >> 2;          // column chunk 32c .. 32c+31
+    const int cg = ew >> 2;         // column group: chunks CPT cg .. CPT cg + CPT - 1
     const int quarter = warp & 3;   // TMEM lanes 32*quarter .. +31
     const int rloc = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -894,38 +752,44 @@ __global__ void __launch_bounds__(kThreadsP, 1)
       }
     }
     const int sw_words = m / 32;  // sign words per vector (2 or 4)
-    // previous tile's row state for the deferred sign readout
+    // previous tile's row state: its signs and residual norm are written one
+    // tile later
     int64_t slot_p = 0;
     bool valid_p = false, zero_p = false;
 
-    // read z of tile Lp (slot parity b) and write this thread's sign word,
-    // then (chunk 0) the residual norm
+    // read z of tile Lp and write this thread's sign word
     auto signs_of = [&](int Lp) -> bool {
       const int b = Lp & 1;
       if (!mbar_wait_warp(smem_u32(&bar_zf[b]), (Lp >> 1) & 1, a.err)) return false;
       tc_fence_after();
-      if (c < sw_words) {
-        uint32_t z[32];
-        tmem_ld32(tmem + (uint32_t)b * 256u + 128u + (uint32_t)(32 * c) + lane_off, z);
-        tmem_ld_wait1(z);
-        uint32_t neg = 0;
 #pragma unroll
-        for (int i = 31; i >= 0; --i) neg = shift_in(neg, z[i]);
-        // bit i = [(S r)_(32c+i) >= 0]; a zero vector's residual was formed
-        // with the opposite sign (see quant32_prod_sb)
-        const uint32_t word = zero_p ? neg : ~neg;
-        if (valid_p) a.signs[slot_p * sw_words + c] = word;
+      for (int cc = 0; cc < CPT; ++cc) {
+        const int c = CPT * cg + cc;
+        if (c < sw_words) {
+          uint32_t z[32];
+          tmem_ld32(tmem + (uint32_t)b * 256u + 128u + (uint32_t)(32 * c) + lane_off, z);
+          tmem_ld_wait1(z);
+          uint32_t neg = 0;
+#pragma unroll
+          for (int i = 31; i >= 0; --i) neg = shift_in(neg, z[i]);
+          // bit i = [(S r)_(32c+i) >= 0]; a zero vector's residual was formed
+          // with the opposite sign (see quant32_prod_sb)
+          const uint32_t word = zero_p ? neg : ~neg;
+          if (valid_p) a.signs[slot_p * sw_words + c] = word;
+        }
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar_zempty[b]));
-      // the partial squares were written before every warp arrived on aready
-      if (c == 0 && !mbar_wait(smem_u32(&bar_aready[b]), (Lp >> 1) & 1, a.err)) return false;
-      if (c == 0 && valid_p) {
-        const float4 q = *reinterpret_cast<const float4*>(&rr_part[b][rloc][0]);
-        a.rnorms[slot_p] = sqrtf((q.x + q.y) + (q.z + q.w)) * (1.0f / 1024.0f);
-      }
+      mbar_arrive(smem_u32(&bar_zempty[b]));
       return true;
+    };
+    // residual norm of the previous tile from the TPR partial squares (the
+    // caller has acquired a barrier that every warp passed after writing them)
+    auto rnorm_of = [&](int Lp) {
+      if (cg == 0 && valid_p) {
+        const float4 q = *reinterpret_cast<const float4*>(&rr_part[Lp & 1][rloc][0]);
+        const float t = TPR == 4 ? (q.x + q.y) + (q.z + q.w) : q.x + q.y;
+        a.rnorms[slot_p] = t > 0.f ? t * rsqrtf(t) * (1.0f / 1024.0f) : 0.f;
+      }
     };
 
     int L = 0;
@@ -936,73 +800,86 @@ __global__ void __launch_bounds__(kThreadsP, 1)
       const int b = L & 1;
       if (!mbar_wait_warp(smem_u32(&bar_accf[b]), (L >> 1) & 1, a.err)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t ucol = tmem + (uint32_t)b * 256u + (uint32_t)(32 * c) + lane_off;
-      uint32_t ur[32];
-      tmem_ld32(ucol, ur);
-      tmem_ld_wait1(ur);
+      const uint32_t ucol = tmem + (uint32_t)b * 256u + (uint32_t)(32 * CPT * cg) + lane_off;
+      uint32_t ur[CPT][32];
+#pragma unroll
+      for (int cc = 0; cc < CPT; ++cc) tmem_ld32(ucol + (uint32_t)(32 * cc), ur[cc]);
+      if (CPT == 2) tmem_ld_wait2(ur[0], ur[CPT - 1]);
+      else tmem_ld_wait1(ur[0]);
       {
         float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const float v0 = __uint_as_float(ur[i]), v1 = __uint_as_float(ur[i + 1]);
-          const float v2 = __uint_as_float(ur[i + 2]), v3 = __uint_as_float(ur[i + 3]);
-          s0 = fmaf(v0, v0, s0);
-          s1 = fmaf(v1, v1, s1);
-          s2 = fmaf(v2, v2, s2);
-          s3 = fmaf(v3, v3, s3);
-        }
-        ss_part[b][rloc][c] = (s0 + s1) + (s2 + s3);
+        for (int cc = 0; cc < CPT; ++cc)
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float v0 = __uint_as_float(ur[cc][i]), v1 = __uint_as_float(ur[cc][i + 1]);
+            const float v2 = __uint_as_float(ur[cc][i + 2]), v3 = __uint_as_float(ur[cc][i + 3]);
+            s0 = fmaf(v0, v0, s0);
+            s1 = fmaf(v1, v1, s1);
+            s2 = fmaf(v2, v2, s2);
+            s3 = fmaf(v3, v3, s3);
+          }
+        ss_part[b][rloc][cg] = (s0 + s1) + (s2 + s3);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar_normx));
+      mbar_arrive(smem_u32(&bar_normx));
       const int64_t row = tile * kRows + rloc;
       const bool valid = row < a.n_vec;
       const int64_t seg = valid ? (int64_t)fastdiv((uint32_t)row, a.seg_div) : 0;
       const int64_t slot = seg * a.seg_cap + (valid ? row - seg * a.seg_len : 0);
       if (!mbar_wait_warp(smem_u32(&bar_normx), (uint32_t)L & 1u, a.err)) { ok = false; break; }
+      // every warp wrote its partials of tile L - 1 before arriving here
+      if (L >= 1) rnorm_of(L - 1);
       const float4 q = *reinterpret_cast<const float4*>(&ss_part[b][rloc][0]);
-      const float nu = sqrtf((q.x + q.y) + (q.z + q.w));  // ||u|| = sqrt(d_pad) ||x||
-      const bool zero = !(nu > 0.f);
-      const float inv = zero ? 0.f : 1024.0f / nu;
-      float v[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ur[i]);
-      uint32_t NS = 0, T0 = 0, T1 = 0, T2 = 0;
+      const float ss = TPR == 4 ? (q.x + q.y) + (q.z + q.w) : q.x + q.y;  // ||u||^2 = d_pad ||x||^2
+      const bool zero = !(ss > 0.f);
+      const float rs = rsqrtf(ss);
+      const float nu = zero ? 0.f : ss * rs;
+      const float inv = zero ? 0.f : 1024.0f * rs;
+      uint32_t NS[CPT], T0[CPT], T1[CPT], T2[CPT];
       float rr = 0.f;
-      quant32_prod_sb<K>(v, tc, dc, c0s, inv, NS, T0, T1, T2, rr);
-      // 2^10 r as fp16 hi (columns 32c .. 32c+15) and lo (32c+16 .. 32c+31)
-      // parts: |r| <= 2, hi keeps the top 11 significant bits (exact in fp16),
-      // lo = 2^10 r - hi is rounded to fp16, about 22 bits in all.
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        uint32_t hiw[8], low[8];
+      for (int cc = 0; cc < CPT; ++cc) {
+        float v[32];
 #pragma unroll
-        for (int qq = 0; qq < 8; ++qq) {
-          const float r0 = v[16 * g + 2 * qq], r1 = v[16 * g + 2 * qq + 1];
-          const float h0 = __uint_as_float(__float_as_uint(r0) & 0xFFFFE000u);
-          const float h1 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
-          const __half2 hv = __floats2half2_rn(h0, h1);
-          const __half2 lv = __floats2half2_rn(r0 - h0, r1 - h1);
-          hiw[qq] = *reinterpret_cast<const uint32_t*>(&hv);
-          low[qq] = *reinterpret_cast<const uint32_t*>(&lv);
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ur[cc][i]);
+        NS[cc] = T0[cc] = T1[cc] = T2[cc] = 0;
+        quant32_prod_sb<K>(v, tc, dc, c0s, inv, NS[cc], T0[cc], T1[cc], T2[cc], rr);
+        // 2^10 r as fp16 hi (columns 32c .. 32c+15) and lo (32c+16 .. 32c+31)
+        // parts: |r| <= 2, hi keeps the top 11 significant bits (exact in
+        // fp16), lo = 2^10 r - hi is rounded to fp16, about 22 bits in all.
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          uint32_t hiw[8], low[8];
+#pragma unroll
+          for (int qq = 0; qq < 8; ++qq) {
+            const float r0 = v[16 * g + 2 * qq], r1 = v[16 * g + 2 * qq + 1];
+            const float h0 = __uint_as_float(__float_as_uint(r0) & 0xFFFFE000u);
+            const float h1 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
+            const __half2 hv = __floats2half2_rn(h0, h1);
+            const __half2 lv = __floats2half2_rn(r0 - h0, r1 - h1);
+            hiw[qq] = *reinterpret_cast<const uint32_t*>(&hv);
+            low[qq] = *reinterpret_cast<const uint32_t*>(&lv);
+          }
+          tmem_st8(ucol + (uint32_t)(32 * cc + 8 * g), hiw);
+          tmem_st8(ucol + (uint32_t)(32 * cc + 16 + 8 * g), low);
         }
-        tmem_st8(ucol + (uint32_t)(8 * g), hiw);
-        tmem_st8(ucol + (uint32_t)(16 + 8 * g), low);
       }
-      rr_part[b][rloc][c] = rr;
+      rr_part[b][rloc][cg] = rr;
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar_aready[b]));
+      mbar_arrive(smem_u32(&bar_aready[b]));
       if (valid) {
-        const uint32_t S = zero ? 0u : ~NS;
-        const uint32_t M0 = K == 3 ? (T0 ^ T1 ^ T2) : T0;
-        uint32_t planes[K];
-        planes_from<K>(S, M0, T1, 0u, planes);
-        uint32_t* dst = a.codes + slot * (int64_t)(K * 4) + c;
+        uint32_t* dst = a.codes + slot * (int64_t)(K * 4) + CPT * cg;
 #pragma unroll
-        for (int p = 0; p < K; ++p) dst[4 * p] = planes[p];
-        if (c == 0) a.norms[slot] = nu * qp.inv_sqrt_dpad;
+        for (int cc = 0; cc < CPT; ++cc) {
+          const uint32_t S = zero ? 0u : ~NS[cc];
+          const uint32_t M0 = K == 3 ? (T0[cc] ^ T1[cc] ^ T2[cc]) : T0[cc];
+          uint32_t planes[K];
+          planes_from<K>(S, M0, T1[cc], 0u, planes);
+#pragma unroll
+          for (int p = 0; p < K; ++p) dst[4 * p + cc] = planes[p];
+        }
+        if (cg == 0) a.norms[slot] = nu * qp.inv_sqrt_dpad;
       }
       // signs of the previous tile: its S r ran while this tile was quantized
       if (L >= 1 && !signs_of(L - 1)) { ok = false; break; }
@@ -1010,7 +887,13 @@ __global__ void __launch_bounds__(kThreadsP, 1)
       valid_p = valid;
       zero_p = zero;
     }
-    if (ok && L >= 1) signs_of(L - 1);
+    if (ok && L >= 1) {
+      // the last tile: its partial squares were written before aready
+      if (mbar_wait_warp(smem_u32(&bar_aready[(L - 1) & 1]), ((L - 1) >> 1) & 1, a.err)) {
+        rnorm_of(L - 1);
+        signs_of(L - 1);
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
