@@ -164,6 +164,44 @@ __device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&r)[32]) {
       : "r"(addr));
 }
 
+// tcgen05.ld of 32 columns and its completion in one statement: the
+// registers are defined only once the data has arrived.
+__device__ __forceinline__ void tmem_ld32_sync(uint32_t addr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(addr)
+      : "memory");
+}
+
+// Packed pairs of fp32 (the f32x2 forms of add, sub and fma).
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 upk2(uint64_t r) {
+  float2 f;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(r));
+  return f;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 // Complete the outstanding tcgen05.ld of this thread; the empty asm
 // statements keep every use of the loaded registers after the wait.
 __device__ __forceinline__ void tmem_ld_wait1(uint32_t (&r)[32]) {
@@ -281,8 +319,8 @@ __device__ __forceinline__ void quant32_mse(const uint32_t (&ur)[32], const floa
 // magnitudes C_j = 2^10 c_j (tc[j] = T_j - C_0, dc[j] = C_(j+1) - C_j).  With
 // e0 = a' - C_0 and d_j = T_j - a', the thermometer bit is sign(d_j), the step
 // [d_j < 0] is exact in {0, 1}, and e = e0 - sum_j step_j dc_j = a' - C_mu.
-// v[i] becomes 2^10 r = +-e with the sign of the coordinate (r = y - C[idx]);
-// rr accumulates (2^10 r)^2.  The sign plane comes from the sign bits of u:
+// v[i] becomes 2^10 r = +-e with the sign of the coordinate (r = y - C[idx]).
+// The sign plane comes from the sign bits of u:
 // NS (bit set = negative) is shifted in and S = ~NS per word.
 // An exactly zero coordinate of a nonzero vector then takes the upper middle
 // cell (a tie at the middle boundary, y = 0 = B); the caller forces S = 0 for
@@ -290,7 +328,7 @@ __device__ __forceinline__ void quant32_mse(const uint32_t (&ur)[32], const floa
 template <int K>
 __device__ __forceinline__ void quant32_prod_sb(float (&v)[32], const float (&tc)[4], const float (&dc)[4],
                                                 float c0, float inv, uint32_t& NS, uint32_t& T0,
-                                                uint32_t& T1, uint32_t& T2, float& rr) {
+                                                uint32_t& T1, uint32_t& T2) {
 #pragma unroll
   for (int i = 31; i >= 0; --i) {
     const uint32_t ub = __float_as_uint(v[i]);
@@ -309,7 +347,6 @@ __device__ __forceinline__ void quant32_prod_sb(float (&v)[32], const float (&tc
         e = fmaf(step_neg(d2), -dc[2], e);
       }
     }
-    rr = fmaf(e, e, rr);
     v[i] = __uint_as_float(__float_as_uint(e) ^ (ub & 0x80000000u));
   }
 }
@@ -767,8 +804,7 @@ __global__ void __launch_bounds__(prod_threads<TPR>(), 1)
         const int c = CPT * cg + cc;
         if (c < sw_words) {
           uint32_t z[32];
-          tmem_ld32(tmem + (uint32_t)b * 256u + 128u + (uint32_t)(32 * c) + lane_off, z);
-          tmem_ld_wait1(z);
+          tmem_ld32_sync(tmem + (uint32_t)b * 256u + 128u + (uint32_t)(32 * c) + lane_off, z);
           uint32_t neg = 0;
 #pragma unroll
           for (int i = 31; i >= 0; --i) neg = shift_in(neg, z[i]);
@@ -803,23 +839,20 @@ __global__ void __launch_bounds__(prod_threads<TPR>(), 1)
       const uint32_t ucol = tmem + (uint32_t)b * 256u + (uint32_t)(32 * CPT * cg) + lane_off;
       uint32_t ur[CPT][32];
 #pragma unroll
-      for (int cc = 0; cc < CPT; ++cc) tmem_ld32(ucol + (uint32_t)(32 * cc), ur[cc]);
-      if (CPT == 2) tmem_ld_wait2(ur[0], ur[CPT - 1]);
-      else tmem_ld_wait1(ur[0]);
+      for (int cc = 0; cc < CPT; ++cc) tmem_ld32_sync(ucol + (uint32_t)(32 * cc), ur[cc]);
       {
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+        uint64_t s2a = 0, s2b = 0;
 #pragma unroll
         for (int cc = 0; cc < CPT; ++cc)
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
-            const float v0 = __uint_as_float(ur[cc][i]), v1 = __uint_as_float(ur[cc][i + 1]);
-            const float v2 = __uint_as_float(ur[cc][i + 2]), v3 = __uint_as_float(ur[cc][i + 3]);
-            s0 = fmaf(v0, v0, s0);
-            s1 = fmaf(v1, v1, s1);
-            s2 = fmaf(v2, v2, s2);
-            s3 = fmaf(v3, v3, s3);
+            const uint64_t p0 = pk2(__uint_as_float(ur[cc][i]), __uint_as_float(ur[cc][i + 1]));
+            const uint64_t p1 = pk2(__uint_as_float(ur[cc][i + 2]), __uint_as_float(ur[cc][i + 3]));
+            s2a = fma2(p0, p0, s2a);
+            s2b = fma2(p1, p1, s2b);
           }
-        ss_part[b][rloc][cg] = (s0 + s1) + (s2 + s3);
+        const float2 fa = upk2(s2a), fb = upk2(s2b);
+        ss_part[b][rloc][cg] = (fa.x + fa.y) + (fb.x + fb.y);
       }
       mbar_arrive(smem_u32(&bar_normx));
       const int64_t row = tile * kRows + rloc;
@@ -836,14 +869,14 @@ __global__ void __launch_bounds__(prod_threads<TPR>(), 1)
       const float nu = zero ? 0.f : ss * rs;
       const float inv = zero ? 0.f : 1024.0f * rs;
       uint32_t NS[CPT], T0[CPT], T1[CPT], T2[CPT];
-      float rr = 0.f;
+      uint64_t rr2 = 0;
 #pragma unroll
       for (int cc = 0; cc < CPT; ++cc) {
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ur[cc][i]);
         NS[cc] = T0[cc] = T1[cc] = T2[cc] = 0;
-        quant32_prod_sb<K>(v, tc, dc, c0s, inv, NS[cc], T0[cc], T1[cc], T2[cc], rr);
+        quant32_prod_sb<K>(v, tc, dc, c0s, inv, NS[cc], T0[cc], T1[cc], T2[cc]);
         // 2^10 r as fp16 hi (columns 32c .. 32c+15) and lo (32c+16 .. 32c+31)
         // parts: |r| <= 2, hi keeps the top 11 significant bits (exact in
         // fp16), lo = 2^10 r - hi is rounded to fp16, about 22 bits in all.
@@ -855,8 +888,11 @@ __global__ void __launch_bounds__(prod_threads<TPR>(), 1)
             const float r0 = v[16 * g + 2 * qq], r1 = v[16 * g + 2 * qq + 1];
             const float h0 = __uint_as_float(__float_as_uint(r0) & 0xFFFFE000u);
             const float h1 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
+            const uint64_t rp = pk2(r0, r1);
+            rr2 = fma2(rp, rp, rr2);
+            const float2 lo = upk2(sub2(rp, pk2(h0, h1)));
             const __half2 hv = __floats2half2_rn(h0, h1);
-            const __half2 lv = __floats2half2_rn(r0 - h0, r1 - h1);
+            const __half2 lv = __floats2half2_rn(lo.x, lo.y);
             hiw[qq] = *reinterpret_cast<const uint32_t*>(&hv);
             low[qq] = *reinterpret_cast<const uint32_t*>(&lv);
           }
@@ -864,6 +900,8 @@ __global__ void __launch_bounds__(prod_threads<TPR>(), 1)
           tmem_st8(ucol + (uint32_t)(32 * cc + 16 + 8 * g), low);
         }
       }
+      const float2 rrf = upk2(rr2);
+      const float rr = rrf.x + rrf.y;
       rr_part[b][rloc][cg] = rr;
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
