@@ -10,6 +10,7 @@
 
 #include "tq_attention.cuh"
 #include "tq_attn2.h"
+#include "tq_attn3.h"
 #include "tq_device.cuh"
 #include "tq_encode.cuh"
 #include "tq_encode2.cuh"
@@ -347,12 +348,17 @@ size_t attention_workspace(const QParams& kp, const QParams& vp, int L, int B, i
   return bytes;
 }
 
-// The tensor-core kernel (tq_attn2.cu) covers d_pad = 128, m = 128, at most 8
-// query heads per KV head and key codes of 1..3 bits; TQ_ATTN_V1=1 selects
-// the SIMT kernel for every shape.
+// The tensor-core kernels (int8: tq_attn3.cu, fp16: tq_attn2.cu) cover
+// d_pad = 128, m = 128, at most 8 query heads per KV head and key codes of
+// 1..3 bits; the int8 kernel runs unless TQ_ATTN_V2=1 selects the fp16 one,
+// and TQ_ATTN_V1=1 selects the SIMT kernel for every shape.
 static const bool g_attn_v2 = [] {
   const char* e = getenv("TQ_ATTN_V1");
   return !(e && e[0] == '1');
+}();
+static const bool g_attn_v3 = [] {
+  const char* e = getenv("TQ_ATTN_V2");
+  return g_attn_v2 && !(e && e[0] == '1');
 }();
 
 static bool attn2_covers(const QParams& kp, const QParams& vp, int G) {
@@ -405,7 +411,8 @@ int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q
     p2.part = part;
     attn2::odd_feature_coefs(kp.centroids, kp.k, p2.kalpha, &p2.kalpha_sum);
     attn2::odd_feature_coefs(vp.centroids, vp.k, p2.valpha, &p2.valpha_sum);
-    cudaError_t ce = attn2::launch(p2, kp.k, vp.k, dim3((unsigned)n_chunks, (unsigned)sh.groups), st);
+    const dim3 grid((unsigned)n_chunks, (unsigned)sh.groups);
+    cudaError_t ce = g_attn_v3 ? attn3::launch(p2, kp.k, vp.k, grid, st) : attn2::launch(p2, kp.k, vp.k, grid, st);
     if (ce != cudaSuccess) return ce;
   } else {
   const size_t smem = (size_t)sh.G * (kp.d_pad + kp.m) * sizeof(float);

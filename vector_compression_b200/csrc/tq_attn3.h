@@ -1,0 +1,18 @@
+// 8-bit integer tensor-core decode attention (tq_attn3.cu): launcher.  Same
+// parameters and partial-output format as the fp16 kernel (tq_attn2.h).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "tq_attn2.h"
+
+namespace tq {
+namespace attn3 {
+
+// d_pad = 128, m = 128, 1..8 query heads per KV head, key codes of 1..3 bits,
+// value codes of 1..4 bits; grid = (chunks, groups), chunks a multiple of 32
+// tokens long.
+cudaError_t launch(const attn2::Params& p, int kk, int kv, dim3 grid, cudaStream_t st);
+
+}  // namespace attn3
+}  // namespace tq
