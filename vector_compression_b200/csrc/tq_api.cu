@@ -409,10 +409,14 @@ int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q
     p2.vcodes = vcodes;
     p2.vnorms = vnorms;
     p2.part = part;
+    p2.err = device_error_ptr();
     attn2::odd_feature_coefs(kp.centroids, kp.k, p2.kalpha, &p2.kalpha_sum);
     attn2::odd_feature_coefs(vp.centroids, vp.k, p2.valpha, &p2.valpha_sum);
     const dim3 grid((unsigned)n_chunks, (unsigned)sh.groups);
-    cudaError_t ce = g_attn_v3 ? attn3::launch(p2, kp.k, vp.k, grid, st) : attn2::launch(p2, kp.k, vp.k, grid, st);
+    // the int8 kernel stages rows with bulk copies: 16-byte aligned arrays
+    const bool v3 = g_attn_v3 && aligned16(ksigns) && aligned16(knorms) && aligned16(krnorms) &&
+                    aligned16(vnorms);
+    cudaError_t ce = v3 ? attn3::launch(p2, kp.k, vp.k, grid, st) : attn2::launch(p2, kp.k, vp.k, grid, st);
     if (ce != cudaSuccess) return ce;
   } else {
   const size_t smem = (size_t)sh.G * (kp.d_pad + kp.m) * sizeof(float);

@@ -23,6 +23,7 @@ struct Params {
   const uint32_t* vcodes;
   const float* vnorms;
   float* part;
+  unsigned* err;    // device error word (bounded waits of the int8 kernel)
   float kalpha[8];  // odd-subset coefficients of the key codebook
   float kalpha_sum;
   float valpha[8];  // and of the value codebook

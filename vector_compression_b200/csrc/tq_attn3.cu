@@ -26,7 +26,10 @@
 // (2^-24 of the largest query entry, 2^-16 of the largest weight).
 //
 // Per CTA: one (layer, batch, kv-head) group and one chunk, 4 warps, in
-// sub-chunks of up to 512 tokens:
+// sub-chunks of up to 512 tokens whose keys, value blocks and norms are
+// staged in shared memory by bulk asynchronous copies (the next sub-chunk's
+// keys load while this one's weights and values are formed, its values while
+// the next scores are):
 //   A. scores: warp w takes 16-token m-tiles w, w + 4, ... (rows = tokens,
 //      K = the 32 coordinates of one plane word, N = heads x {hi, lo}); the
 //      scores go to shared memory, with the sub-chunk maximum per head;
@@ -79,7 +82,9 @@ __device__ __forceinline__ void mma_u8u8(int (&d)[4], uint32_t a0, uint32_t a1, 
 // Bytes {0, 128} from bits s0 + 8 i (i = 0..3) of w, mul = 2^(7 - s0): the
 // multiply moves them to the byte sign positions.
 __device__ __forceinline__ uint32_t bits_to_bytes(uint32_t w, uint32_t mul) {
-  return (w * mul) & 0x80808080u;
+  uint32_t r;  // an integer multiply (FMA pipe), not a shift (ALU pipe)
+  asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(mul));
+  return r & 0x80808080u;
 }
 
 template <int K>
@@ -115,16 +120,77 @@ __device__ __forceinline__ uint32_t fixed_byte(float x, float inv, int piece) {
   return (uint32_t)((piece == 0 ? hi : piece == 1 ? mid : lo) & 0xFF);
 }
 
+// Shared-memory layout of one CTA (bytes): the staged sub-chunk (key codes,
+// sign words, key norms, residual norms | value blocks, value norms), scores,
+// weight bytes, and the query rows used during setup.
+template <int KK, int KV, int NT>
+struct Layout {
+  static constexpr int KW = KK * WPP, HN = 4 * NT;
+  static constexpr uint32_t kc = 0;
+  static constexpr uint32_t ks = kc + SC * KW * 4;
+  static constexpr uint32_t kn = ks + SC * SW * 4;
+  static constexpr uint32_t kr = kn + SC * 4;
+  static constexpr uint32_t vc = kr + SC * 4;
+  static constexpr uint32_t vn = vc + (SC / 32) * KV * DP * 4;
+  static constexpr uint32_t score = vn + SC * 4;
+  static constexpr uint32_t wb = score + SC * HN * 4;
+  static constexpr uint32_t qf = wb + (SC / 32) * NT * 8 * 4 * 2 * 4;
+  static constexpr uint32_t bytes = qf + 2 * HN * DP * 4;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from
+// global to shared memory, completing on the mbarrier.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// Bounded wait for the phase with the given parity (suspend-hinted); false
+// and the device error word set if it does not complete within ~2^31 cycles.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity), "r"(20000u)
+        : "memory");
+    if (done) return true;
+    if (clock64() - t0 > (1LL << 31)) {
+      if (err) atomicCAS(err, 0u, (unsigned)TQ_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 template <int KK, int KV, int NT>
 __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
+  using LY = Layout<KK, KV, NT>;
   constexpr int FK = NF<KK>::v;  // key code features
   constexpr int FV = NF<KV>::v;  // value code features
   constexpr int KW = KK * WPP;   // key code words per token
   constexpr int HN = 4 * NT;     // head slots
+  constexpr float kLog2e = 1.4426950408889634f;
 
-  __shared__ float s_score[SC][HN];  // scores, then weights p ||v||
-  __shared__ __align__(16) uint32_t s_wb[SC / 32][NT][8][4][2];  // weight bytes, B-fragment order
-  __shared__ float s_qf[2][HN][DP];  // q' and u (M = DP) of the heads
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint32_t* s_kc = reinterpret_cast<uint32_t*>(smem + LY::kc);   // [SC][KW]
+  uint32_t* s_ks = reinterpret_cast<uint32_t*>(smem + LY::ks);   // [SC][SW]
+  float* s_kn = reinterpret_cast<float*>(smem + LY::kn);         // [SC]
+  float* s_kr = reinterpret_cast<float*>(smem + LY::kr);         // [SC]
+  uint32_t* s_vc = reinterpret_cast<uint32_t*>(smem + LY::vc);   // [SC/32][KV*DP]
+  float* s_vn = reinterpret_cast<float*>(smem + LY::vn);         // [SC]
+  float (*s_score)[HN] = reinterpret_cast<float (*)[HN]>(smem + LY::score);  // log2-domain scores, then weights
+  uint32_t (*s_wb)[NT][8][4][2] = reinterpret_cast<uint32_t (*)[NT][8][4][2]>(smem + LY::wb);
+  float (*s_qf)[HN][DP] = reinterpret_cast<float (*)[HN][DP]>(smem + LY::qf);
+  __shared__ __align__(8) uint64_t bar_k, bar_v;
   __shared__ float s_red[3][kWarps][HN];
   __shared__ float s_head[HN][8];  // per head: Qq, Qu, sum q_int, sum u_int, m, l, 1/Qq, 1/Qu
 
@@ -132,8 +198,40 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
   const int g = lane >> 2, tig = lane & 3;
   const int G = P.G;
   const int grp = blockIdx.y, chunk = blockIdx.x;
+  const int64_t t_begin = (int64_t)chunk * P.chunk;
+  const int64_t t_end = min64(P.seq, t_begin + P.chunk);
+  const int64_t krow0 = (int64_t)grp * P.cap;
+  const int64_t vblk0 = (int64_t)grp * (P.cap / 32);
   // K slots 4 tig + i <-> bits 2 tig + 8 i, 16 + 4 tig + i <-> bits 2 tig + 1 + 8 i
   const uint32_t mul0 = 1u << (7 - 2 * tig), mul1 = 1u << (6 - 2 * tig);
+
+  // ---- staging of sub-chunks (one thread issues the bulk copies)
+  const uint32_t bk = smem_u32(&bar_k), bv = smem_u32(&bar_v);
+  // keys of the sub-chunk at s: codes, signs, norms, residual norms of
+  // round_up(n, 4) tokens (inside the cache: cap >= round_up(seq, 32))
+  auto issue_keys = [&](int64_t s) {
+    const uint32_t n4 = (uint32_t)((min64(SC, t_end - s) + 3) & ~3);
+    mbar_expect(bk, n4 * (KW * 4 + SW * 4 + 8));
+    bulk_g2s(s_kc, P.kcodes + (krow0 + s) * KW, n4 * KW * 4, bk);
+    bulk_g2s(s_ks, P.ksigns + (krow0 + s) * SW, n4 * SW * 4, bk);
+    bulk_g2s(s_kn, P.knorms + krow0 + s, n4 * 4, bk);
+    bulk_g2s(s_kr, P.krnorms + krow0 + s, n4 * 4, bk);
+  };
+  // values of the sub-chunk at s: its 32-token blocks and the value norms
+  auto issue_values = [&](int64_t s) {
+    const int64_t n = min64(SC, t_end - s);
+    const uint32_t nb = (uint32_t)((n + 31) / 32), n4 = (uint32_t)((n + 3) & ~3);
+    mbar_expect(bv, nb * KV * DP * 4 + n4 * 4);
+    bulk_g2s(s_vc, P.vcodes + (vblk0 + s / 32) * (int64_t)(KV * DP), nb * KV * DP * 4, bv);
+    bulk_g2s(s_vn, P.vnorms + krow0 + s, n4 * 4, bv);
+  };
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bk));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bv));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    issue_keys(t_begin);
+    issue_values(t_begin);
+  }
 
   // ---- query side: fixed-point scales and the score B fragments
   for (int e = tid; e < 2 * HN * DP; e += kThreads) {
@@ -162,7 +260,7 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
     }
   }
   if (tid < HN) {
-    s_head[tid][4] = -INFINITY;  // running max
+    s_head[tid][4] = -INFINITY;  // running max (log2 domain)
     s_head[tid][5] = 0.f;        // running sum of p
   }
   __syncthreads();
@@ -193,55 +291,54 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
       }
     }
   }
-  // per thread-column heads (4 nt + tig): score constants
+  // per thread-column heads (4 nt + tig): score constants, log2 domain
   float cA1[NT], cC1[NT], cA2[NT], cC2[NT];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int h = 4 * nt + tig;
     const float Qq = s_head[h][0], Qu = s_head[h][1];
-    cA1[nt] = Qq * (1.0f / 64.0f);                // <q', b> = Qq v / 128, times 2
-    cC1[nt] = -Qq * P.kalpha_sum * s_head[h][2];  // - sum_S alpha_S sum q'
-    cA2[nt] = P.kappa * Qu * (1.0f / 64.0f);
-    cC2[nt] = -P.kappa * Qu * s_head[h][3];
+    const float sl = P.scale * kLog2e;
+    cA1[nt] = sl * Qq * (1.0f / 64.0f);                // <q', b> = Qq v / 128, times 2
+    cC1[nt] = -sl * Qq * P.kalpha_sum * s_head[h][2];  // - sum_S alpha_S sum q'
+    cA2[nt] = sl * P.kappa * Qu * (1.0f / 64.0f);
+    cC2[nt] = -sl * P.kappa * Qu * s_head[h][3];
   }
 
-  const int64_t t_begin = (int64_t)chunk * P.chunk;
-  const int64_t t_end = min64(P.seq, t_begin + P.chunk);
-  const int64_t krow0 = (int64_t)grp * P.cap;
-  const int64_t vblk0 = (int64_t)grp * (P.cap / 32);
-  const float scale = P.scale;
   float o_run[NT][2][2];  // [nt][jh][row]: coordinate 32 warp + 16 jh + g + 8 row, head 4 nt + tig
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int jh = 0; jh < 2; ++jh) o_run[nt][jh][0] = o_run[nt][jh][1] = 0.f;
 
-  for (int64_t s0 = t_begin; s0 < t_end; s0 += SC) {
+  uint32_t phase = 0;
+  bool ok = true;
+  for (int64_t s0 = t_begin; s0 < t_end; s0 += SC, phase ^= 1u) {
     const int scn = (int)min64(SC, t_end - s0);  // tokens of this sub-chunk
-    // ================= A. scores
+    // ================= A. scores (log2 domain) from the staged keys
+    bool okw = mbar_wait(bk, phase, P.err);
     float mloc[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) mloc[nt] = -INFINITY;
-    for (int mt = warp; 16 * mt < scn; mt += kWarps) {
+    for (int mt = warp; okw && 16 * mt < scn; mt += kWarps) {
       const int l1 = 16 * mt + g, l2 = l1 + 8;
       const bool ok1 = l1 < scn, ok2 = l2 < scn;
-      const int64_t R1 = krow0 + s0 + (ok1 ? l1 : scn - 1), R2 = krow0 + s0 + (ok2 ? l2 : scn - 1);
+      const int R1 = ok1 ? l1 : scn - 1, R2 = ok2 ? l2 : scn - 1;
       uint32_t k1[KW + SW], k2[KW + SW];
 #pragma unroll
       for (int i = 0; i < KW; i += 4) {
-        const uint4 a = *reinterpret_cast<const uint4*>(P.kcodes + R1 * KW + i);
-        const uint4 b = *reinterpret_cast<const uint4*>(P.kcodes + R2 * KW + i);
+        const uint4 a = *reinterpret_cast<const uint4*>(s_kc + R1 * KW + i);
+        const uint4 b = *reinterpret_cast<const uint4*>(s_kc + R2 * KW + i);
         k1[i] = a.x; k1[i + 1] = a.y; k1[i + 2] = a.z; k1[i + 3] = a.w;
         k2[i] = b.x; k2[i + 1] = b.y; k2[i + 2] = b.z; k2[i + 3] = b.w;
       }
       {
-        const uint4 a = *reinterpret_cast<const uint4*>(P.ksigns + R1 * SW);
-        const uint4 b = *reinterpret_cast<const uint4*>(P.ksigns + R2 * SW);
+        const uint4 a = *reinterpret_cast<const uint4*>(s_ks + R1 * SW);
+        const uint4 b = *reinterpret_cast<const uint4*>(s_ks + R2 * SW);
         k1[KW] = a.x; k1[KW + 1] = a.y; k1[KW + 2] = a.z; k1[KW + 3] = a.w;
         k2[KW] = b.x; k2[KW + 1] = b.y; k2[KW + 2] = b.z; k2[KW + 3] = b.w;
       }
-      const float n1 = P.knorms[R1], n2 = P.knorms[R2];
-      const float r1 = P.krnorms[R1], r2 = P.krnorms[R2];
+      const float n1 = s_kn[R1], n2 = s_kn[R2];
+      const float r1 = s_kr[R1], r2 = s_kr[R2];
       int acc[FK + 1][NT + 1][4];
 #pragma unroll
       for (int f = 0; f <= FK; ++f)
@@ -268,11 +365,12 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
             mma_u8s8(acc[f][nt], a0, a1, a2, a3, bq[nt][which][cw][0], bq[nt][which][cw][1]);
         }
       }
-      // s = scale n (Qq (sum_S alpha_S v_S / 64 - sum alpha sum q_int)
-      //              + kappa rho Qu (v_sign / 64 - sum u_int)),
-      // v = 2^16 hi + 2^8 mid + lo (hi, mid: tile nt; lo: tile NT, column nt)
+      // s log2(e) = scale log2(e) n (Qq (sum_S alpha_S v_S / 64 - sum alpha sum q_int)
+      //                     + kappa rho Qu (v_sign / 64 - sum u_int)),
+      // v = 2^16 hi + 2^8 mid + lo (hi, mid: tile nt; lo: tile NT, column nt);
+      // 2^8 hi + mid stays below 2^31.
       auto comb = [&](const int (&t)[NT + 1][4], int nt, int row) {
-        return fmaf(65536.f, (float)t[nt][2 * row], fmaf(256.f, (float)t[nt][2 * row + 1], (float)t[NT][2 * row + nt]));
+        return fmaf(256.f, (float)(256 * t[nt][2 * row] + t[nt][2 * row + 1]), (float)t[NT][2 * row + nt]);
       };
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -285,8 +383,8 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
         }
         const float q1 = comb(acc[FK], nt, 0);
         const float q2 = comb(acc[FK], nt, 1);
-        const float x1 = scale * n1 * (fmaf(cA1[nt], m1, cC1[nt]) + r1 * fmaf(cA2[nt], q1, cC2[nt]));
-        const float x2 = scale * n2 * (fmaf(cA1[nt], m2, cC1[nt]) + r2 * fmaf(cA2[nt], q2, cC2[nt]));
+        const float x1 = n1 * (fmaf(cA1[nt], m1, cC1[nt]) + r1 * fmaf(cA2[nt], q1, cC2[nt]));
+        const float x2 = n2 * (fmaf(cA1[nt], m2, cC1[nt]) + r2 * fmaf(cA2[nt], q2, cC2[nt]));
         if (h < G) {
           if (ok1) s_score[l1][h] = x1;
           if (ok2) s_score[l2][h] = x2;
@@ -303,9 +401,12 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
       if (g == 0) s_red[0][warp][4 * nt + tig] = v;
     }
-    __syncthreads();
-    // ================= B. weights
-    // thread tid: tokens tid, tid + 128, ... of the sub-chunk, every head
+    ok = __syncthreads_and(okw) != 0;
+    if (!ok) break;
+    // the key buffer is free: stage the next sub-chunk's keys
+    if (tid == 0 && s0 + SC < t_end) issue_keys(s0 + SC);
+    // ================= B. weights p ||v||, p = 2^(s - m)
+    okw = mbar_wait(bv, phase, P.err);
     float mnew[HN], lpart[HN], wmax[HN];
 #pragma unroll
     for (int h = 0; h < HN; ++h) {
@@ -316,13 +417,12 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
       lpart[h] = 0.f;
       wmax[h] = 0.f;
     }
-    for (int t = tid; t < scn; t += kThreads) {
-      const float vn = P.vnorms[krow0 + s0 + t];
+    for (int t = tid; okw && t < scn; t += kThreads) {
+      const float vn = s_vn[t];
 #pragma unroll
       for (int h = 0; h < HN; ++h) {
         if (h < G) {
-          const float s = s_score[t][h];
-          const float p = s == -INFINITY ? 0.f : expf(s - mnew[h]);
+          const float p = exp2f(s_score[t][h] - mnew[h]);
           const float w = p * vn;
           s_score[t][h] = w;
           lpart[h] += p;
@@ -332,13 +432,14 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
     }
 #pragma unroll
     for (int h = 0; h < HN; ++h) {
-      float a = warp_sum(lpart[h]), b = warp_max(wmax[h]);
+      const float a = warp_sum(lpart[h]), b = warp_max(wmax[h]);
       if (lane == 0) {
         s_red[1][warp][h] = a;
         s_red[2][warp][h] = b;
       }
     }
-    __syncthreads();
+    ok = __syncthreads_and(okw) != 0;
+    if (!ok) break;
     float winv[HN];
 #pragma unroll
     for (int h = 0; h < HN; ++h) {
@@ -386,14 +487,15 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
         wi = hh == h ? winv[hh] : wi;
       }
       const float mold = s_head[h][4];
-      corr[nt] = mold == -INFINITY ? 0.f : expf(mold - mn);
+      corr[nt] = mold == -INFINITY ? 0.f : exp2f(mold - mn);
       wscale[nt] = wi > 0.f ? 1.0f / wi : 0.f;
       int ws = 0;
 #pragma unroll
       for (int v = 0; v < kWarps; ++v) ws += __float_as_int(s_red[0][v][h]);
       wtot[nt] = (float)ws;
     }
-    // ================= C. values: coordinates 32 warp + 16 jh + g + 8 row
+    // ================= C. values from the staged blocks: coordinates
+    // 32 warp + 16 jh + g + 8 row
     int accv[FV][2][NT][4];
 #pragma unroll
     for (int f = 0; f < FV; ++f)
@@ -402,7 +504,7 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) accv[f][jh][nt][0] = accv[f][jh][nt][1] = accv[f][jh][nt][2] = accv[f][jh][nt][3] = 0;
     for (int blk = 0; 32 * blk < scn; ++blk) {
-      const uint32_t* vw = P.vcodes + (vblk0 + s0 / 32 + blk) * (int64_t)(KV * DP);
+      const uint32_t* vw = s_vc + blk * (KV * DP);
       uint32_t pw[2][2][KV];
 #pragma unroll
       for (int jh = 0; jh < 2; ++jh)
@@ -434,16 +536,17 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
       for (int jh = 0; jh < 2; ++jh) {
 #pragma unroll
         for (int rw = 0; rw < 2; ++rw) {
-          float s = 0.f;
+          float sv = 0.f;
 #pragma unroll
           for (int f = 0; f < FV; ++f)
-            s = fmaf(P.valpha[f], fmaf(256.f, (float)accv[f][jh][nt][2 * rw], (float)accv[f][jh][nt][2 * rw + 1]), s);
-          const float o_sub = wscale[nt] * fmaf(s, 1.0f / 64.0f, -P.valpha_sum * wtot[nt]);
+            sv = fmaf(P.valpha[f], fmaf(256.f, (float)accv[f][jh][nt][2 * rw], (float)accv[f][jh][nt][2 * rw + 1]), sv);
+          const float o_sub = wscale[nt] * fmaf(sv, 1.0f / 64.0f, -P.valpha_sum * wtot[nt]);
           o_run[nt][jh][rw] = fmaf(o_run[nt][jh][rw], corr[nt], o_sub);
         }
       }
     }
-    __syncthreads();  // every thread has read s_head / s_red / s_wb of this sub-chunk
+    __syncthreads();  // every thread has read s_head, s_red, s_wb and the value buffer
+    if (tid == 0 && s0 + SC < t_end) issue_values(s0 + SC);
     if (tid < HN && tid < G) {
       float ls = 0.f, mn = 0.f;
 #pragma unroll
@@ -451,14 +554,22 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
 #pragma unroll
       for (int hh = 0; hh < HN; ++hh) mn = hh == tid ? mnew[hh] : mn;
       const float mold = s_head[tid][4];
-      const float c = mold == -INFINITY ? 0.f : expf(mold - mn);
+      const float c = mold == -INFINITY ? 0.f : exp2f(mold - mn);
       s_head[tid][5] = s_head[tid][5] * c + ls;
       s_head[tid][4] = mn;
     }
     __syncthreads();
   }
+  if (!ok) {
+    // a staging wait expired (error word set): let copies still in flight land
+    if (tid == 0) {
+      mbar_wait(bk, phase, nullptr);
+      mbar_wait(bv, phase, nullptr);
+    }
+    return;
+  }
 
-  // ---- partial (m, l, o_rot) of this chunk
+  // ---- partial (m, l, o_rot) of this chunk (m back in the natural-log domain)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int h = 4 * nt + tig;
@@ -469,19 +580,25 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
 #pragma unroll
       for (int rw = 0; rw < 2; ++rw) pp[2 + 32 * warp + 16 * jh + g + 8 * rw] = o_run[nt][jh][rw];
     if (warp == 0 && g == 0) {
-      pp[0] = s_head[h][4];
+      pp[0] = s_head[h][4] * (1.0f / kLog2e);
       pp[1] = s_head[h][5];
     }
   }
 }
 
+template <int KK, int KV, int NT>
+cudaError_t launch_nt(const Params& p, dim3 grid, cudaStream_t st) {
+  auto kern = attn_kernel<KK, KV, NT>;
+  const int smem = (int)Layout<KK, KV, NT>::bytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
 template <int KK, int KV>
 cudaError_t launch_kv(const Params& p, dim3 grid, cudaStream_t st) {
-  if (p.G <= 4)
-    attn_kernel<KK, KV, 1><<<grid, kThreads, 0, st>>>(p);
-  else
-    attn_kernel<KK, KV, 2><<<grid, kThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return p.G <= 4 ? launch_nt<KK, KV, 1>(p, grid, st) : launch_nt<KK, KV, 2>(p, grid, st);
 }
 
 template <int KK>
