@@ -59,7 +59,7 @@ constexpr int DP = 128;            // rotated dimension
 constexpr int WPP = DP / 32;       // words per code plane
 constexpr int M = 128;             // QJL rows
 constexpr int SW = M / 32;         // sign words per token
-constexpr int SC = 512;            // tokens per sub-chunk
+constexpr int SC = 384;            // tokens per sub-chunk (a multiple of 64)
 constexpr float kQMax = 8323072.0f;  // 127 * 2^16: the hi byte stays in [-127, 127]
 
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -121,8 +121,8 @@ __device__ __forceinline__ uint32_t fixed_byte(float x, float inv, int piece) {
 }
 
 // Shared-memory layout of one CTA (bytes): the staged sub-chunk (key codes,
-// sign words, key norms, residual norms | value blocks, value norms), scores,
-// weight bytes, and the query rows used during setup.
+// sign words, key norms, residual norms | value blocks, value norms), scores
+// (which first hold the query rows during setup) and weight bytes.
 template <int KK, int KV, int NT>
 struct Layout {
   static constexpr int KW = KK * WPP, HN = 4 * NT;
@@ -134,8 +134,10 @@ struct Layout {
   static constexpr uint32_t vn = vc + (SC / 32) * KV * DP * 4;
   static constexpr uint32_t score = vn + SC * 4;
   static constexpr uint32_t wb = score + SC * HN * 4;
-  static constexpr uint32_t qf = wb + (SC / 32) * NT * 8 * 4 * 2 * 4;
-  static constexpr uint32_t bytes = qf + 2 * HN * DP * 4;
+  static constexpr uint32_t bytes = wb + (SC / 32) * NT * 8 * 4 * 2 * 4;
+  // the query rows (setup only) share the score buffer
+  static constexpr uint32_t qf = score;
+  static_assert(SC * HN >= 2 * HN * DP, "query rows fit in the score buffer");
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -188,6 +190,7 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
   uint32_t* s_vc = reinterpret_cast<uint32_t*>(smem + LY::vc);   // [SC/32][KV*DP]
   float* s_vn = reinterpret_cast<float*>(smem + LY::vn);         // [SC]
   float (*s_score)[HN] = reinterpret_cast<float (*)[HN]>(smem + LY::score);  // log2-domain scores, then weights
+  static_assert(LY::score % 16 == 0, "vector access to the score rows");
   uint32_t (*s_wb)[NT][8][4][2] = reinterpret_cast<uint32_t (*)[NT][8][4][2]>(smem + LY::wb);
   float (*s_qf)[HN][DP] = reinterpret_cast<float (*)[HN][DP]>(smem + LY::qf);
   __shared__ __align__(8) uint64_t bar_k, bar_v;
@@ -291,6 +294,7 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
       }
     }
   }
+  __syncthreads();  // the query rows (in the score buffer) have been read
   // per thread-column heads (4 nt + tig): score constants, log2 domain
   float cA1[NT], cC1[NT], cA2[NT], cC2[NT];
 #pragma unroll
@@ -420,14 +424,19 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
     for (int t = tid; okw && t < scn; t += kThreads) {
       const float vn = s_vn[t];
 #pragma unroll
-      for (int h = 0; h < HN; ++h) {
-        if (h < G) {
-          const float p = exp2f(s_score[t][h] - mnew[h]);
+      for (int h4 = 0; h4 < HN; h4 += 4) {
+        float4 sc4 = *reinterpret_cast<const float4*>(&s_score[t][h4]);
+        float* sc = reinterpret_cast<float*>(&sc4);
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh) {
+          const int h = h4 + hh;
+          const float p = h < G ? exp2f(sc[hh] - mnew[h]) : 0.f;
           const float w = p * vn;
-          s_score[t][h] = w;
+          sc[hh] = w;
           lpart[h] += p;
           wmax[h] = fmaxf(wmax[h], w);
         }
+        *reinterpret_cast<float4*>(&s_score[t][h4]) = sc4;
       }
     }
 #pragma unroll
@@ -457,10 +466,19 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
     for (int t = tid; t < scn32; t += kThreads) {
       const int blk = t >> 5, tau = t & 31;
       const int tg = (tau & 7) >> 1, r = tau & 1, i = tau >> 3;
+      float wrow[HN];
+#pragma unroll
+      for (int h4 = 0; h4 < HN; h4 += 4) {
+        const float4 w4 = t < scn ? *reinterpret_cast<const float4*>(&s_score[t][h4]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        wrow[h4] = w4.x;
+        wrow[h4 + 1] = w4.y;
+        wrow[h4 + 2] = w4.z;
+        wrow[h4 + 3] = w4.w;
+      }
 #pragma unroll
       for (int h = 0; h < HN; ++h) {
         if (h < G) {
-          const int wi = t < scn ? __float2int_rn(s_score[t][h] * winv[h]) : 0;
+          const int wi = __float2int_rn(wrow[h] * winv[h]);
           wsum[h] += wi;
           unsigned char* hb = reinterpret_cast<unsigned char*>(&s_wb[blk][h >> 2][2 * (h & 3)][tg][r]);
           unsigned char* lb = reinterpret_cast<unsigned char*>(&s_wb[blk][h >> 2][2 * (h & 3) + 1][tg][r]);
