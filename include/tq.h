@@ -295,6 +295,36 @@ tq_status tq_decode_attention_noalloc(const tq_params* kp, const tq_params* vp, 
                                       void* stream);
 
 /*
+ * tq_decode_step -- one serving decode step over a compressed KV cache:
+ * append the new token's key and value to every (layer, batch, kv-head)
+ * cache at slot `pos`, then attend over the pos + 1 cached tokens
+ * ("turboquant-pytorch" skill page, KV Cache Wrapper (TurboQuantKVCache):
+ * append_key / append_value as tokens are generated, then attention of a
+ * query against all cached keys with MSE-reconstructed values).
+ *   k_new, v_new DEVICE [L][B][Hkv][d] of dtype dt (rows 16-byte aligned):
+ *           the new token's key and value per (layer, batch, kv-head)
+ *   pos     slot of the new token, 0 <= pos < cap; slots 0 .. pos - 1 must
+ *           already hold the earlier tokens (e.g. from tq_encode_prod /
+ *           tq_encode_mse or earlier steps)
+ *   kcodes, ksigns, knorms, krnorms, vcodes, vnorms  the caches of
+ *           tq_decode_attention, written at slot pos (in BLOCK32 only bit
+ *           pos % 32 of block pos / 32 changes) and then read
+ *   q, Hq, Hkv, cap, scale, out  as tq_decode_attention with seq = pos + 1
+ *   ws      workspace of tq_decode_step_workspace_size bytes (256-byte
+ *           aligned)
+ * Everything is enqueued on `stream` in order (key encode, value encode,
+ * bit scatter, attention).  Errors: those of tq_decode_attention, and
+ * TQ_ERR_INVALID_ARG for pos outside [0, cap) or a bad dtype.
+ */
+tq_status tq_decode_step(const tq_params* kp, const tq_params* vp, const float* q,
+                         const void* k_new, const void* v_new, tq_dtype dt, int L, int B, int Hq,
+                         int Hkv, int64_t pos, int64_t cap, float scale, uint32_t* kcodes,
+                         uint32_t* ksigns, float* knorms, float* krnorms, uint32_t* vcodes,
+                         float* vnorms, float* out, void* ws, size_t ws_bytes, void* stream);
+tq_status tq_decode_step_workspace_size(const tq_params* kp, const tq_params* vp, int L, int B,
+                                        int Hq, int Hkv, int64_t pos, size_t* bytes);
+
+/*
  * tq_sync_check -- synchronize `stream` and report (then clear) the device
  * error word that kernels set when a bounded wait expires (TQ_ERR_TIMEOUT)
  * or an internal check fails (TQ_ERR_INTERNAL).

@@ -281,6 +281,34 @@ def tq_decode_attention_noalloc(kp: TQParams, vp: TQParams, q, kcache, vcache, s
     return out
 
 
+def tq_decode_step(kp: TQParams, vp: TQParams, q, k_new, v_new, kcache, vcache, pos: int, cap: int,
+                   scale: float, out=None, ws=None, stream=None):
+    """One serving decode step: append k_new / v_new [L, B, Hkv, d] (fp32, fp16
+    or bf16) at slot pos of the caches (updated in place), then attend q
+    [L, B, Hq, d] over the pos + 1 cached tokens.  Returns out [L, B, Hq, d]."""
+    torch = _torch()
+    Ln, B, Hq, d = q.shape
+    kcodes, ksigns, knorms, krnorms = kcache
+    vcodes, vnorms = vcache
+    Hkv = k_new.shape[2]
+    if k_new.dtype != v_new.dtype or k_new.shape != v_new.shape or k_new.shape != (Ln, B, Hkv, d):
+        raise ValueError("k_new and v_new must be [L, B, Hkv, d] of one dtype")
+    kn, vn = k_new.contiguous(), v_new.contiguous()
+    if out is None:
+        out = torch.empty((Ln, B, Hq, d), dtype=torch.float32, device=q.device)
+    need = C.c_size_t()
+    L.check("tq_decode_step_workspace_size", L.lib().tq_decode_step_workspace_size(
+        kp.handle, vp.handle, Ln, B, Hq, Hkv, pos, C.byref(need)))
+    if ws is None or ws.numel() < need.value:
+        ws = _ws(need.value, q.device)
+    qc = q.contiguous()
+    L.check("tq_decode_step", L.lib().tq_decode_step(
+        kp.handle, vp.handle, _ptr(qc), _ptr(kn), _ptr(vn), _dtype_code(kn), Ln, B, Hq, Hkv, pos, cap,
+        float(scale), _ptr(kcodes), _ptr(ksigns), _ptr(knorms), _ptr(krnorms), _ptr(vcodes),
+        _ptr(vnorms), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
 def tq_sync_check(stream=None):
     """Synchronize and raise if a kernel flagged a device-side error."""
     L.check("tq_sync_check", L.lib().tq_sync_check(_stream(stream)))

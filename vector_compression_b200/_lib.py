@@ -42,6 +42,9 @@ SIGNATURES = {
                                  _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "tq_decode_attention_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i64, _i64, _f,
                                          _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "tq_decode_step_workspace_size": (_i, [_vp, _vp, _i, _i, _i, _i, _i64, C.POINTER(_sz)]),
+    "tq_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64, _i64, _f,
+                            _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "tq_sync_check": (_i, [_vp]),
 }
 
