@@ -314,6 +314,10 @@ def main():
         if ent and ent.get("source_hash") == source_hash():
             traffic = ent["bytes_per_launch"]
 
+    # ---- serving decode step (outside the timed region): append the last
+    # token of every (layer, batch, kv-head) at slot seq - 1 and attend
+    step_info = decode_step_timing(tq, kp, vp, K, V, q, kc, vcodes, vnorms, out, seq, cap, scale, stream)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -350,6 +354,7 @@ def main():
             "e2e": None if e2e is None else {"value": e2e["value"], "unit": UNIT,
                                              "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
             "cpu_baseline": cpu,
+            "decode_step": step_info,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -365,6 +370,31 @@ def source_hash():
     for f in sorted(os.listdir(csrc)):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
+
+
+def decode_step_timing(tq, kp, vp, K, V, q, kc, vcodes, vnorms, out, seq, cap, scale, stream, reps=10):
+    """Latency of tq_decode_step on the full cache: the new token of every
+    (layer, batch, kv-head) is the cache's last row, appended at slot seq - 1
+    (rewriting it with the same codes), then attention over seq tokens."""
+    import torch
+
+    kn = K[:, :, :, seq - 1].contiguous()
+    vn = V[:, :, :, seq - 1].contiguous()
+    L_, B, Hkv = kn.shape[0], kn.shape[1], kn.shape[2]
+    ws = torch.empty(tq.tq_decode_step_workspace_size(kp, vp, L_, B, q.shape[2], Hkv, seq - 1),
+                     dtype=torch.uint8, device=q.device)
+    for _ in range(3):
+        tq.tq_decode_step(kp, vp, q, kn, vn, kc, (vcodes, vnorms), seq - 1, cap, scale, out=out, ws=ws)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        tq.tq_decode_step(kp, vp, q, kn, vn, kc, (vcodes, vnorms), seq - 1, cap, scale, out=out, ws=ws)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    return {"ms": ms, "tokens_appended": int(L_ * B * Hkv), "context": seq, "launches": 6}
 
 
 def run_e2e(args, tq, kp, vp, K, V, q, kc, vcodes, vnorms, out, ws, seq, cap, scale, step_bytes):

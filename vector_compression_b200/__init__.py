@@ -281,6 +281,14 @@ def tq_decode_attention_noalloc(kp: TQParams, vp: TQParams, q, kcache, vcache, s
     return out
 
 
+def tq_decode_step_workspace_size(kp: TQParams, vp: TQParams, L_: int, B: int, Hq: int, Hkv: int,
+                                  pos: int) -> int:
+    need = C.c_size_t()
+    L.check("tq_decode_step_workspace_size", L.lib().tq_decode_step_workspace_size(
+        kp.handle, vp.handle, L_, B, Hq, Hkv, pos, C.byref(need)))
+    return need.value
+
+
 def tq_decode_step(kp: TQParams, vp: TQParams, q, k_new, v_new, kcache, vcache, pos: int, cap: int,
                    scale: float, out=None, ws=None, stream=None):
     """One serving decode step: append k_new / v_new [L, B, Hkv, d] (fp32, fp16
@@ -296,11 +304,9 @@ def tq_decode_step(kp: TQParams, vp: TQParams, q, k_new, v_new, kcache, vcache, 
     kn, vn = k_new.contiguous(), v_new.contiguous()
     if out is None:
         out = torch.empty((Ln, B, Hq, d), dtype=torch.float32, device=q.device)
-    need = C.c_size_t()
-    L.check("tq_decode_step_workspace_size", L.lib().tq_decode_step_workspace_size(
-        kp.handle, vp.handle, Ln, B, Hq, Hkv, pos, C.byref(need)))
-    if ws is None or ws.numel() < need.value:
-        ws = _ws(need.value, q.device)
+    need = tq_decode_step_workspace_size(kp, vp, Ln, B, Hq, Hkv, pos)
+    if ws is None or ws.numel() < need:
+        ws = _ws(need, q.device)
     qc = q.contiguous()
     L.check("tq_decode_step", L.lib().tq_decode_step(
         kp.handle, vp.handle, _ptr(qc), _ptr(kn), _ptr(vn), _dtype_code(kn), Ln, B, Hq, Hkv, pos, cap,
