@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-groups", type=int, default=6)
+    ap.add_argument("--qjl-rows", type=int, default=0,
+                    help="QJL projection rows m of the keys (0 = the padded head dim; d_pad / 2 is the half-size variant)")
     return ap.parse_args()
 
 
@@ -139,7 +141,7 @@ class OracleSample:
     (layer, batch, kv-head) groups of one layer, each fully encoded (keys
     Q_prod, values Q_MSE) and attended by its G query heads."""
 
-    def __init__(self, cfg, groups: int, layer: int = 0):
+    def __init__(self, cfg, groups: int, layer: int = 0, m: int = 0):
         import torch
 
         from oracle import tq_oracle as o
@@ -148,7 +150,7 @@ class OracleSample:
         self.cfg = cfg
         torch.set_num_threads(max(1, os.cpu_count() or 1))
         self.cores = torch.get_num_threads()
-        kd = synth.method_draws(cfg.head_dim, cfg.d_pad, cfg.seed, stream=1)
+        kd = synth.method_draws(cfg.head_dim, m or cfg.d_pad, cfg.seed, stream=1)
         vd = synth.method_draws(cfg.head_dim, cfg.d_pad, cfg.seed, stream=2)
         self.kq = o.Quantizer(cfg.head_dim, cfg.key_bits, prod=True, draws=kd)
         self.vq = o.Quantizer(cfg.head_dim, cfg.value_bits, prod=False, draws=vd)
@@ -181,7 +183,7 @@ def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    sample = OracleSample(cfg, max(1, args.cpu_sample_groups // 3))
+    sample = OracleSample(cfg, max(1, args.cpu_sample_groups // 3), m=args.qjl_rows)
     for _ in range(args.warmup):
         sample.run()
     vals, secs = [], []
@@ -227,9 +229,10 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
-    kd = synth.method_draws(cfg.head_dim, cfg.d_pad, cfg.seed, stream=1)
+    m = args.qjl_rows or cfg.d_pad
+    kd = synth.method_draws(cfg.head_dim, m, cfg.seed, stream=1)
     vd = synth.method_draws(cfg.head_dim, cfg.d_pad, cfg.seed, stream=2)
-    kp = tq.TQParams(cfg.head_dim, cfg.key_bits, tq.MODE_PROD, tq.ROT_HADAMARD, m=cfg.d_pad,
+    kp = tq.TQParams(cfg.head_dim, cfg.key_bits, tq.MODE_PROD, tq.ROT_HADAMARD, m=m,
                      signs=kd["signs"], S=kd["S"])
     vp = tq.TQParams(cfg.head_dim, cfg.value_bits, tq.MODE_MSE, tq.ROT_HADAMARD, signs=vd["signs"])
     K, V = synth.kv_cache(cfg, device=dev)
@@ -331,7 +334,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1:
-        s = OracleSample(cfg, args.cpu_sample_groups)
+        s = OracleSample(cfg, args.cpu_sample_groups, m=args.qjl_rows)
         v, dt = s.run()
         cpu = {"value": v, "unit": UNIT, "cores": s.cores, "kind": "oracle", "sample": s.sample, "seconds": dt}
 

@@ -4,7 +4,7 @@ attention over the grown sequence, and at the end every cache slot holds
 the oracle's codes of the original key/value rows (slots past the sequence
 untouched).  Covers a prefill of 70 tokens plus three steps, block
 boundaries (pos 31, 32), the first token of an empty cache and the last slot,
-d = 192 (256-point rotation) with 8 query heads per KV head, and argument
+m = 64 QJL rows, d = 192 (256-point rotation) with 8 query heads per KV head, and argument
 errors."""
 import math
 
@@ -22,8 +22,8 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def make_pair(d, bits, prod, seed, stream):
-    m = synth.next_pow2(d)
+def make_pair(d, bits, prod, seed, stream, m=None):
+    m = m or synth.next_pow2(d)
     dr = synth.method_draws(d, m, seed, stream=stream)
     ora = o.Quantizer(d, bits, prod=prod, draws=dr)
     lib = tq.TQParams(d, bits, tq.MODE_PROD if prod else tq.MODE_MSE, tq.ROT_HADAMARD,
@@ -62,10 +62,10 @@ def check_cache(kq, vq, K, V, kc, vc, n_tok, cap):
             assert np.all((tail[t // 32] >> np.uint32(t % 32)) & 1 == 0)
 
 
-def run_steps(d, G, bits, cap, prefill, steps, dtype="float16", seed=7):
+def run_steps(d, G, bits, cap, prefill, steps, dtype="float16", seed=7, m=None):
     Ln, B, Hkv = 2, 1, 2
     groups = Ln * B * Hkv
-    kq, kl = make_pair(d, bits, True, seed, 1)
+    kq, kl = make_pair(d, bits, True, seed, 1, m=m)
     vq, vl = make_pair(d, bits, False, seed, 2)
     T = prefill + steps
     rng = np.random.default_rng(seed)
@@ -113,6 +113,11 @@ def test_decode_steps_cross_block_boundary():
 def test_decode_steps_from_empty_to_last_slot():
     run_steps(128, 1, 2, cap=32, prefill=0, steps=3, dtype="float32")
     run_steps(128, 2, 4, cap=32, prefill=29, steps=3)
+
+
+def test_decode_steps_qjl_half_rows():
+    # QJL with m = d / 2 = 64 projection rows
+    run_steps(128, 4, 3, cap=96, prefill=62, steps=3, m=64)
 
 
 def test_decode_steps_d192_gqa8():

@@ -208,12 +208,16 @@ def _pack_cache(ora_k, ora_v, K, V, seq, cap):
     return (t(kc), t(ks), t(kn), t(kr)), (t(vc), t(vn)), encs
 
 
-@pytest.mark.parametrize("d,G,seq,cap,bits", [(128, 8, 300, 320, 3), (128, 4, 64, 64, 2),
-                                              (192, 4, 1000, 1024, 4), (128, 1, 33, 64, 3)])
-def test_attention_on_oracle_cache(d, G, seq, cap, bits):
+@pytest.mark.parametrize("d,G,seq,cap,bits,m", [(128, 8, 300, 320, 3, None), (128, 4, 64, 64, 2, None),
+                                                (192, 4, 1000, 1024, 4, None), (128, 1, 33, 64, 3, None),
+                                                (128, 4, 1000, 1024, 3, 64), (128, 8, 97, 128, 2, 64),
+                                                (128, 2, 413, 416, 4, 64)])
+def test_attention_on_oracle_cache(d, G, seq, cap, bits, m):
+    # m = 64: the QJL projection with d / 2 rows (a storage variant with
+    # 8 bytes of signs per token instead of 16)
     Ln, B, Hkv = 2, 1, 2
     Hq = G * Hkv
-    kq, kl = make_pair(d, bits, True, seed=40, stream=1)
+    kq, kl = make_pair(d, bits, True, seed=40, m=m, stream=1)
     vq, vl = make_pair(d, bits, False, seed=40, stream=2)
     rng = np.random.default_rng(5)
     K = rng.standard_normal((Ln * B * Hkv, seq, d)) * rng.lognormal(0, 1, size=(1, 1, d))
@@ -231,7 +235,7 @@ def test_attention_on_oracle_cache(d, G, seq, cap, bits):
                 want = o.decode_attention(q[l, b, h * G:(h + 1) * G], kq, vq, ke, ve, scale, G)
                 got = out[l, b, h * G:(h + 1) * G]
                 err = np.linalg.norm(got - want, axis=1) / np.linalg.norm(want, axis=1)
-                print(f"attention rel err (G={G}, bits={bits}): {err.max():.2e}")
+                print(f"attention rel err (G={G}, bits={bits}, m={kq.m}): {err.max():.2e}")
                 assert err.max() <= REL_TOL, err.max()
 
 

@@ -361,9 +361,11 @@ static const bool g_attn_v3 = [] {
   return g_attn_v2 && !(e && e[0] == '1');
 }();
 
+// m = 128 for the fp16 kernel; the int8 kernel also takes m = 64
 static bool attn2_covers(const QParams& kp, const QParams& vp, int G) {
   return g_attn_v2 && kp.rot == TQ_ROT_HADAMARD && kp.d_pad == 128 && vp.d_pad == 128 &&
-         kp.m == 128 && G >= 1 && G <= 8 && kp.k >= 1 && kp.k <= 3 && vp.k >= 1 && vp.k <= 4;
+         (kp.m == 128 || (kp.m == 64 && g_attn_v3)) && G >= 1 && G <= 8 && kp.k >= 1 && kp.k <= 3 &&
+         vp.k >= 1 && vp.k <= 4;
 }
 
 int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q, int L, int B,
@@ -416,7 +418,11 @@ int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q
     // the int8 kernel stages rows with bulk copies: 16-byte aligned arrays
     const bool v3 = g_attn_v3 && aligned16(ksigns) && aligned16(knorms) && aligned16(krnorms) &&
                     aligned16(vnorms);
-    cudaError_t ce = v3 ? attn3::launch(p2, kp.k, vp.k, grid, st) : attn2::launch(p2, kp.k, vp.k, grid, st);
+    cudaError_t ce = cudaErrorInvalidValue;
+    if (v3)
+      ce = attn3::launch(p2, kp.k, vp.k, kp.m, grid, st);
+    else if (kp.m == 128)
+      ce = attn2::launch(p2, kp.k, vp.k, grid, st);
     if (ce != cudaSuccess) return ce;
   } else {
   const size_t smem = (size_t)sh.G * (kp.d_pad + kp.m) * sizeof(float);

@@ -57,8 +57,6 @@ constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
 constexpr int DP = 128;            // rotated dimension
 constexpr int WPP = DP / 32;       // words per code plane
-constexpr int M = 128;             // QJL rows
-constexpr int SW = M / 32;         // sign words per token
 constexpr int SC = 384;            // tokens per sub-chunk (a multiple of 64)
 constexpr float kQMax = 8323072.0f;  // 127 * 2^16: the hi byte stays in [-127, 127]
 
@@ -123,9 +121,9 @@ __device__ __forceinline__ uint32_t fixed_byte(float x, float inv, int piece) {
 // Shared-memory layout of one CTA (bytes): the staged sub-chunk (key codes,
 // sign words, key norms, residual norms | value blocks, value norms), scores
 // (which first hold the query rows during setup) and weight bytes.
-template <int KK, int KV, int NT>
+template <int KK, int KV, int NT, int MQ>
 struct Layout {
-  static constexpr int KW = KK * WPP, HN = 4 * NT;
+  static constexpr int KW = KK * WPP, HN = 4 * NT, SW = MQ / 32;
   static constexpr uint32_t kc = 0;
   static constexpr uint32_t ks = kc + SC * KW * 4;
   static constexpr uint32_t kn = ks + SC * SW * 4;
@@ -173,9 +171,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   }
 }
 
-template <int KK, int KV, int NT>
+template <int KK, int KV, int NT, int MQ>
 __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
-  using LY = Layout<KK, KV, NT>;
+  using LY = Layout<KK, KV, NT, MQ>;
+  constexpr int SW = MQ / 32;    // QJL sign words per token (m = 64 or 128)
   constexpr int FK = NF<KK>::v;  // key code features
   constexpr int FV = NF<KV>::v;  // value code features
   constexpr int KW = KK * WPP;   // key code words per token
@@ -240,7 +239,8 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
   for (int e = tid; e < 2 * HN * DP; e += kThreads) {
     const int which = e / (HN * DP), h = (e / DP) % HN, j = e % DP;
     float x = 0.f;
-    if (h < G) x = which == 0 ? P.qrot[((int64_t)grp * G + h) * DP + j] : P.u[((int64_t)grp * G + h) * M + j];
+    if (h < G && (which == 0 || j < MQ))
+      x = which == 0 ? P.qrot[((int64_t)grp * G + h) * DP + j] : P.u[((int64_t)grp * G + h) * MQ + j];
     s_qf[which][h][j] = x;
   }
   for (int e = tid; e < (SC / 32) * NT * 8 * 4 * 2; e += kThreads) (&s_wb[0][0][0][0][0])[e] = 0u;
@@ -335,11 +335,16 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
         k1[i] = a.x; k1[i + 1] = a.y; k1[i + 2] = a.z; k1[i + 3] = a.w;
         k2[i] = b.x; k2[i + 1] = b.y; k2[i + 2] = b.z; k2[i + 3] = b.w;
       }
-      {
+      if (SW == 4) {
         const uint4 a = *reinterpret_cast<const uint4*>(s_ks + R1 * SW);
         const uint4 b = *reinterpret_cast<const uint4*>(s_ks + R2 * SW);
         k1[KW] = a.x; k1[KW + 1] = a.y; k1[KW + 2] = a.z; k1[KW + 3] = a.w;
         k2[KW] = b.x; k2[KW + 1] = b.y; k2[KW + 2] = b.z; k2[KW + 3] = b.w;
+      } else {
+        const uint2 a = *reinterpret_cast<const uint2*>(s_ks + R1 * SW);
+        const uint2 b = *reinterpret_cast<const uint2*>(s_ks + R2 * SW);
+        k1[KW] = a.x; k1[KW + 1] = a.y;
+        k2[KW] = b.x; k2[KW + 1] = b.y;
       }
       const float n1 = s_kn[R1], n2 = s_kn[R2];
       const float r1 = s_kr[R1], r2 = s_kr[R2];
@@ -358,6 +363,7 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
         }
 #pragma unroll
         for (int f = 0; f <= FK; ++f) {
+          if (f == FK && cw >= SW) continue;  // the sign plane has m / 32 words
           // features of the key code, then the QJL sign plane
           const uint32_t W1 = f < FK ? feature_word<KK>(p1, f) : k1[KW + cw];
           const uint32_t W2 = f < FK ? feature_word<KK>(p2, f) : k2[KW + cw];
@@ -604,10 +610,10 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
   }
 }
 
-template <int KK, int KV, int NT>
+template <int KK, int KV, int NT, int MQ>
 cudaError_t launch_nt(const Params& p, dim3 grid, cudaStream_t st) {
-  auto kern = attn_kernel<KK, KV, NT>;
-  const int smem = (int)Layout<KK, KV, NT>::bytes;
+  auto kern = attn_kernel<KK, KV, NT, MQ>;
+  const int smem = (int)Layout<KK, KV, NT, MQ>::bytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, st>>>(p);
@@ -615,27 +621,28 @@ cudaError_t launch_nt(const Params& p, dim3 grid, cudaStream_t st) {
 }
 
 template <int KK, int KV>
-cudaError_t launch_kv(const Params& p, dim3 grid, cudaStream_t st) {
-  return p.G <= 4 ? launch_nt<KK, KV, 1>(p, grid, st) : launch_nt<KK, KV, 2>(p, grid, st);
+cudaError_t launch_kv(const Params& p, int m, dim3 grid, cudaStream_t st) {
+  if (m == 64) return p.G <= 4 ? launch_nt<KK, KV, 1, 64>(p, grid, st) : launch_nt<KK, KV, 2, 64>(p, grid, st);
+  return p.G <= 4 ? launch_nt<KK, KV, 1, 128>(p, grid, st) : launch_nt<KK, KV, 2, 128>(p, grid, st);
 }
 
 template <int KK>
-cudaError_t launch_k(const Params& p, int kv, dim3 grid, cudaStream_t st) {
+cudaError_t launch_k(const Params& p, int kv, int m, dim3 grid, cudaStream_t st) {
   switch (kv) {
-    case 1: return launch_kv<KK, 1>(p, grid, st);
-    case 2: return launch_kv<KK, 2>(p, grid, st);
-    case 3: return launch_kv<KK, 3>(p, grid, st);
-    case 4: return launch_kv<KK, 4>(p, grid, st);
+    case 1: return launch_kv<KK, 1>(p, m, grid, st);
+    case 2: return launch_kv<KK, 2>(p, m, grid, st);
+    case 3: return launch_kv<KK, 3>(p, m, grid, st);
+    case 4: return launch_kv<KK, 4>(p, m, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch(const Params& p, int kk, int kv, dim3 grid, cudaStream_t st) {
-  if (p.G < 1 || p.G > 8) return cudaErrorInvalidValue;
+cudaError_t launch(const Params& p, int kk, int kv, int m, dim3 grid, cudaStream_t st) {
+  if (p.G < 1 || p.G > 8 || (m != 64 && m != 128)) return cudaErrorInvalidValue;
   switch (kk) {
-    case 1: return launch_k<1>(p, kv, grid, st);
-    case 2: return launch_k<2>(p, kv, grid, st);
-    case 3: return launch_k<3>(p, kv, grid, st);
+    case 1: return launch_k<1>(p, kv, m, grid, st);
+    case 2: return launch_k<2>(p, kv, m, grid, st);
+    case 3: return launch_k<3>(p, kv, m, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
