@@ -39,6 +39,12 @@ DESIGN.md):
 * QJL scale sqrt(pi/2)/m with m rows of S ([EXPL] §8 has m = d).
 * The residual and S act in the rotated domain ([EXPL] §8: r = Pi x - y_mse).
 * A zero vector has norm 0 and is encoded from the zero rotated vector.
+* Unbiased per-vector scale (EDEN; DRIVE at one bit): the Q_MSE codes are
+  kept and the stored scale is S = ||x||^2 / <Pi x, C[idx]> = n / <y, C[idx]>
+  in place of n, so that the unchanged decoder n Pi^T C[idx] becomes
+  S Pi^T C[idx].  The codebook stays the Beta(d_pad) one (TurboQuant is EDEN
+  with the scale fixed; the pages' decoder-split discussion).  A vector with
+  <y, C[idx]> = 0 (only the zero vector) stores 0.
 
 Every function below has a pin in ``tests/test_oracle_pins.py``.
 """
@@ -363,10 +369,12 @@ class Quantizer:
     definition of Q_prod).
     """
 
-    def __init__(self, d: int, bits: int, *, prod: bool, draws: dict):
+    def __init__(self, d: int, bits: int, *, prod: bool, draws: dict, unbiased: bool = False):
         self.d = d
         self.bits = bits
         self.prod = prod
+        # Q_MSE with EDEN's unbiased per-vector scale in place of the norm
+        self.unbiased = bool(unbiased) and not prod
         self.k = bits - 1 if prod else bits
         if draws.get("G") is not None:
             self.rot = Rotation(d, G=draws["G"])
@@ -407,6 +415,8 @@ class Quantizer:
         n, y = self.rotate_unit(x)
         idx = self.quantize(y)
         out = {"norms": n.astype(np.float32), "idx": idx, "y": y}
+        if self.unbiased:
+            out["norms"] = self.unbiased_scale(n, y, idx).astype(np.float32)
         pack = pack_row if layout == "row" else pack_block32
         out["codes"] = pack(idx, self.k)
         if self.prod:
@@ -418,6 +428,17 @@ class Quantizer:
             sig = (z >= 0).astype(np.int64)
             out.update(rnorms=rho.astype(np.float32), signs=pack_signs(sig), z=z, rho64=rho)
         return out
+
+    def unbiased_scale(self, n, y, idx):
+        """EDEN's per-vector scale ([EXPL] prior work, EDEN paragraph:
+        S = ||x||^2 / <R(x), Q(R(x))>, which makes S R^T Q(R(x)) unbiased; DRIVE
+        is the one-bit case, S = ||x||^2 / ||R(x)||_1 with sign codes).  Here
+        R(x) = Pi x = n y and Q(R(x)) = n C[idx] up to the codebook's fixed
+        scale, which cancels between the scale and the decoder:
+        S = n^2 / (n <y, C[idx]>) = n / <y, C[idx]>."""
+        dot = np.sum(y * self.centroids[idx], axis=-1)
+        ok = dot > 0
+        return np.where(ok, np.asarray(n, np.float64) / np.where(ok, dot, 1.0), 0.0)
 
     # -- decode / estimate -------------------------------------------------
 

@@ -341,6 +341,70 @@ def test_qmse_shrinkage_over_haar_rotations():
     assert abs(lam - 2 / math.pi) < 0.02
 
 
+# ---------------------------------------------------------------- unbiased (EDEN / DRIVE) scale
+
+
+@pytest.mark.parametrize("d,bits,dense", [(24, 1, True), (24, 3, True), (100, 2, False),
+                                          (128, 4, False), (192, 3, False)])
+def test_unbiased_scale_keeps_the_component_along_x(d, bits, dense):
+    # x~ = S Pi^T C[idx] with S = ||x||^2 / <Pi x, C[idx]> (EDEN's scale): the
+    # component of x~ along x is x itself for every rotation, <x~, x> = ||x||^2,
+    # up to the fp32 rounding of the stored scale.  The plain norm (Q_MSE) or
+    # the least-squares scale n <y, C> / ||C||^2 both miss it.
+    rng = np.random.default_rng(51)
+    q = o.Quantizer(d, bits, prod=False, draws=_draws(d, 32, 3, dense=dense), unbiased=True)
+    x = rng.standard_normal((200, d)) * rng.lognormal(0, 1, size=(200, 1))
+    x[7] = 0.0
+    e = q.encode(x)
+    xt = q.decode(e["idx"], e["norms"])
+    got, want = np.sum(xt * x, axis=1), np.sum(x * x, axis=1)
+    nz = want > 0
+    assert np.max(np.abs(got[nz] / want[nz] - 1.0)) < 3e-7
+    assert e["norms"][7] == 0.0 and np.all(xt[7] == 0.0)
+    plain = o.Quantizer(d, bits, prod=False, draws=_draws(d, 32, 3, dense=dense))
+    pe = plain.encode(x)
+    assert np.array_equal(pe["idx"], e["idx"])  # same codes, only the scale differs
+    xp = plain.decode(pe["idx"], pe["norms"])
+    assert np.min(np.abs(np.sum(xp * x, axis=1)[nz] / want[nz] - 1.0)) > 1e-4
+
+
+@pytest.mark.parametrize("dense", [True, False])
+def test_unbiased_scale_one_bit_is_drive(dense):
+    # One bit: C[idx] = +-c1 sign(y), and the scale reduces to DRIVE's unbiased
+    # S = ||x||^2 / ||R x||_1 applied to sign(R x): x~ = S R^T sign(R x), with R
+    # written out here as an explicit matrix.
+    rng = np.random.default_rng(52)
+    d = 40
+    q = o.Quantizer(d, 1, prod=False, draws=_draws(d, 32, 4, dense=dense), unbiased=True)
+    R = q.rot.apply(np.eye(d)).T  # column i = R e_i
+    x = rng.standard_normal((50, d)) * 2.5
+    e = q.encode(x)
+    xt = q.decode(e["idx"], e["norms"])
+    Rx = x @ R.T
+    S = np.sum(x * x, axis=1) / np.sum(np.abs(Rx), axis=1)
+    drive = S[:, None] * (np.sign(Rx) @ R)
+    np.testing.assert_allclose(xt, drive, rtol=3e-7, atol=3e-7 * np.abs(drive).max())
+
+
+def test_unbiased_scale_over_haar_rotations():
+    # EDEN: over uniformly random rotations the reconstruction is unbiased,
+    # E[x~] = x (each coordinate within 4 standard errors), where the plain
+    # norm shrinks it by lambda_b.
+    rng = np.random.default_rng(61)
+    d, bits, n = 16, 2, 10000
+    x = rng.standard_normal(d)
+    xs = np.empty((n, d))
+    for s in range(n):
+        dr = {"signs": None, "S": None, "G": np.random.default_rng([61, s]).standard_normal((d, d))}
+        q = o.Quantizer(d, bits, prod=False, draws=dr, unbiased=True)
+        e = q.encode(x[None])
+        xs[s] = q.decode(e["idx"], e["norms"])[0]
+    se = xs.std(axis=0) / math.sqrt(n)
+    assert np.all(np.abs(xs.mean(axis=0) - x) < 4 * se)
+    lam = o.shrinkage(d, bits)
+    assert np.any(np.abs(lam * x - x) > 8 * se)  # the test separates the biased decoder
+
+
 def test_residual_norm_expectation():
     # Residual energy: E||r||^2 = d_pad * C(f, b-1) over random unit inputs
     # (the notes' E||r|| = sqrt(C) read as the second moment); dense Haar
