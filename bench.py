@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-groups", type=int, default=6)
+    ap.add_argument("--value-scale", default="norm", choices=["norm", "unbiased"],
+                    help="per-vector scale stored with the values: the norm, or EDEN's unbiased scale")
     ap.add_argument("--qjl-rows", type=int, default=0,
                     help="QJL projection rows m of the keys (0 = the padded head dim; d_pad / 2 is the half-size variant)")
     return ap.parse_args()
@@ -141,7 +143,7 @@ class OracleSample:
     (layer, batch, kv-head) groups of one layer, each fully encoded (keys
     Q_prod, values Q_MSE) and attended by its G query heads."""
 
-    def __init__(self, cfg, groups: int, layer: int = 0, m: int = 0):
+    def __init__(self, cfg, groups: int, layer: int = 0, m: int = 0, unbiased: bool = False):
         import torch
 
         from oracle import tq_oracle as o
@@ -153,7 +155,7 @@ class OracleSample:
         kd = synth.method_draws(cfg.head_dim, m or cfg.d_pad, cfg.seed, stream=1)
         vd = synth.method_draws(cfg.head_dim, cfg.d_pad, cfg.seed, stream=2)
         self.kq = o.Quantizer(cfg.head_dim, cfg.key_bits, prod=True, draws=kd)
-        self.vq = o.Quantizer(cfg.head_dim, cfg.value_bits, prod=False, draws=vd)
+        self.vq = o.Quantizer(cfg.head_dim, cfg.value_bits, prod=False, draws=vd, unbiased=unbiased)
         one = cfg.scaled(layers=1)
         K, V = synth.kv_cache(one, device="cpu", layers=range(layer, layer + 1))
         q = synth.decode_queries(one, device="cpu", layers=range(layer, layer + 1))
@@ -183,7 +185,8 @@ def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    sample = OracleSample(cfg, max(1, args.cpu_sample_groups // 3), m=args.qjl_rows)
+    sample = OracleSample(cfg, max(1, args.cpu_sample_groups // 3), m=args.qjl_rows,
+                          unbiased=args.value_scale == "unbiased")
     for _ in range(args.warmup):
         sample.run()
     vals, secs = [], []
@@ -234,7 +237,8 @@ def main():
     vd = synth.method_draws(cfg.head_dim, cfg.d_pad, cfg.seed, stream=2)
     kp = tq.TQParams(cfg.head_dim, cfg.key_bits, tq.MODE_PROD, tq.ROT_HADAMARD, m=m,
                      signs=kd["signs"], S=kd["S"])
-    vp = tq.TQParams(cfg.head_dim, cfg.value_bits, tq.MODE_MSE, tq.ROT_HADAMARD, signs=vd["signs"])
+    vmode = tq.MODE_MSE_UNBIASED if args.value_scale == "unbiased" else tq.MODE_MSE
+    vp = tq.TQParams(cfg.head_dim, cfg.value_bits, vmode, tq.ROT_HADAMARD, signs=vd["signs"])
     K, V = synth.kv_cache(cfg, device=dev)
     q = synth.decode_queries(cfg, device=dev)
     seq = cap = cfg.seq
@@ -334,7 +338,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1:
-        s = OracleSample(cfg, args.cpu_sample_groups, m=args.qjl_rows)
+        s = OracleSample(cfg, args.cpu_sample_groups, m=args.qjl_rows, unbiased=args.value_scale == "unbiased")
         v, dt = s.run()
         cpu = {"value": v, "unit": UNIT, "cores": s.cores, "kind": "oracle", "sample": s.sample, "seconds": dt}
 
@@ -345,7 +349,7 @@ def main():
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": cfg.name, "layers": cfg.layers, "batch": cfg.batch, "kv_heads": cfg.kv_heads,
                        "q_heads": cfg.q_heads, "head_dim": cfg.head_dim, "seq": cfg.seq, "input_dtype": cfg.dtype,
-                       "key_bits": cfg.key_bits, "value_bits": cfg.value_bits, "qjl_m": kp.m,
+                       "key_bits": cfg.key_bits, "value_bits": cfg.value_bits, "qjl_m": kp.m, "value_scale": args.value_scale,
                        "rotation": "randomized Hadamard", "l2": "inputs larger than L2 (no flush)",
                        "bytes_per_step": step_bytes, "parallelism": f"replica x{world}"},
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["GB/s"], "peak": peak,

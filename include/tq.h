@@ -63,7 +63,7 @@ typedef enum {
 
 typedef enum { TQ_F32 = 0, TQ_F16 = 1, TQ_BF16 = 2 } tq_dtype;
 typedef enum { TQ_ROT_HADAMARD = 0, TQ_ROT_DENSE = 1 } tq_rot;
-typedef enum { TQ_MODE_MSE = 0, TQ_MODE_PROD = 1 } tq_mode;
+typedef enum { TQ_MODE_MSE = 0, TQ_MODE_PROD = 1, TQ_MODE_MSE_UNBIASED = 2 } tq_mode;
 typedef enum { TQ_LAYOUT_ROW = 0, TQ_LAYOUT_BLOCK32 = 1 } tq_layout;
 
 typedef struct tq_params tq_params; /* opaque quantizer description */
@@ -107,7 +107,16 @@ tq_status tq_make_rotation(int d, const double* G, float* Pi);
  *   bits    total bit budget b per coordinate: Q_MSE uses b-bit codes
  *           (1..4); Q_prod uses (b-1)-bit codes plus one QJL sign per row of
  *           S (b = 2..5) ([EXPL] §8, [NOTES] definition of Q_prod)
- *   mode    TQ_MODE_MSE or TQ_MODE_PROD
+ *   mode    TQ_MODE_MSE, TQ_MODE_PROD or TQ_MODE_MSE_UNBIASED.  The last
+ *           writes the same b-bit codes as TQ_MODE_MSE but stores, in place
+ *           of the norm n = ||x||, EDEN's unbiased per-vector scale
+ *           S = ||x||^2 / <Pi x, C[idx]> = n / <y, C[idx]> ([EXPL] prior
+ *           work: EDEN's scale, and DRIVE's ||x||^2 / ||Pi x||_1 at b = 1),
+ *           0 for a zero vector.  Every Q_MSE decoder (tq_decode, the value
+ *           side of tq_decode_attention / tq_decode_step) then reconstructs
+ *           S Pi^T C[idx], whose component along x is exactly x and whose
+ *           mean over uniformly random rotations is x.  Accepted wherever
+ *           TQ_MODE_MSE is.
  *   rot     TQ_ROT_HADAMARD: Pi = H D / sqrt(d_pad), d_pad = next power of
  *           two >= d (at least 32), the vector zero-padded ([EXPL] §0.9,
  *           [FVQ]); d_pad must be 32..256.

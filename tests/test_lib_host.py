@@ -88,6 +88,19 @@ def test_params_validation():
     assert lib.tq_params_create(128, 3, 1, 0, 100, p, S.ctypes.data_as(C.c_void_p), None, C.byref(h)) == 1
     S = np.full((128, 128), 0.1, np.float32)  # not fp16-representable
     assert lib.tq_params_create(128, 3, 1, 0, 128, p, S.ctypes.data_as(C.c_void_p), None, C.byref(h)) == 1
+    assert lib.tq_params_create(128, 3, 3, 0, 0, p, None, None, C.byref(h)) == 1    # no mode 3
+
+
+def test_unbiased_mode_handle():
+    # Q_MSE with the unbiased (EDEN) scale: same code geometry as Q_MSE, and
+    # accepted by the Q_MSE entry points' validation (a Q_prod call is not)
+    u = tq.TQParams(128, 2, tq.MODE_MSE_UNBIASED, tq.ROT_HADAMARD, signs=np.ones(128, np.int8))
+    assert (u.d_pad, u.k, u.code_words, u.sign_words, u.m) == (128, 2, 8, 0, 0)
+    lib = L.lib()
+    fake = C.c_void_p(0x10000)
+    assert lib.tq_encode_mse(u.handle, fake, 0, 0, 128, 0, 0, 0, None, None, None, 0, None) == 0  # empty
+    assert lib.tq_encode_mse(u.handle, None, 0, 10, 128, 0, 0, 0, fake, fake, None, 0, None) == 1
+    assert lib.tq_encode_prod(u.handle, fake, 0, 10, 128, 0, 0, fake, fake, fake, fake, None, 0, None) == 1
 
 
 def test_encode_and_attention_validation_before_launch():

@@ -14,7 +14,7 @@ from typing import Optional
 import numpy as np
 
 from . import _lib as L
-from ._lib import (BF16, F16, F32, LAYOUT_BLOCK32, LAYOUT_ROW, MODE_MSE, MODE_PROD,  # noqa: F401
+from ._lib import (BF16, F16, F32, LAYOUT_BLOCK32, LAYOUT_ROW, MODE_MSE, MODE_MSE_UNBIASED, MODE_PROD,  # noqa: F401
                    ROT_DENSE, ROT_HADAMARD, TQError)
 
 __all__ = [

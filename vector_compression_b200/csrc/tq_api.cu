@@ -103,7 +103,7 @@ cudaError_t encode_dense(const QParams& qp, bool prod, const T* x, int64_t ld, i
     cudaError_t e = gemm_abt_f32(xh, qp.Pi, y, (int)rows, d, d, st);
     if (e != cudaSuccess) return e;
     quantize_rows_kernel<<<(unsigned)ceil_div(ceil_div(rows, 32), 4), 128, 0, st>>>(
-        qp, y, seg_len, seg_cap, row, rows, layout, prod, codes, rnorms);
+        qp, y, seg_len, seg_cap, row, rows, layout, prod, codes, norms, rnorms);
     if (prod) {
       e = gemm_abt_f32(y, qp.S, z, (int)rows, qp.m, d, st);
       if (e != cudaSuccess) return e;
@@ -176,7 +176,10 @@ bool try_encode_v2(const QParams& qp, bool prod, const void* x, int dt, int64_t 
   const int64_t want = ceil_div(a.n_tasks, 4);
   const int resident = (smem <= 113 * 1024) ? 2 : 1;
   const int ctas = (int)std::min<int64_t>(want, (int64_t)num_sms() * resident);
-  const int mode = prod ? enc2::MODE_PROD : (layout == TQ_LAYOUT_BLOCK32 ? enc2::MODE_MSE_BLOCK : enc2::MODE_MSE_ROW);
+  const bool blk = layout == TQ_LAYOUT_BLOCK32;
+  const int mode = prod ? enc2::MODE_PROD
+                        : qp.unbiased ? (blk ? enc2::MODE_MSE_BLOCK_U : enc2::MODE_MSE_ROW_U)
+                                      : (blk ? enc2::MODE_MSE_BLOCK : enc2::MODE_MSE_ROW);
   a.err = device_error_ptr();
   if (!a.err) return false;
   cudaError_t e;
@@ -528,7 +531,7 @@ tq_status tq_encode_mse(const tq_params* p, const void* x, tq_dtype dt, int64_t 
                         float* norms, void* ws, size_t ws_bytes, void* stream) {
   tq_status s = check_encode_common(p, x, dt, n_vec, ld, &seg_len, &seg_cap, layout);
   if (s != TQ_OK) return s;
-  if (p->mode != TQ_MODE_MSE) return TQ_ERR_INVALID_ARG;
+  if (p->mode != TQ_MODE_MSE && p->mode != TQ_MODE_MSE_UNBIASED) return TQ_ERR_INVALID_ARG;
   if (n_vec == 0) return TQ_OK;
   if (!codes || !norms || !tq::aligned16(codes) || !tq::aligned16(norms)) return TQ_ERR_INVALID_ARG;
   const size_t need = tq::encode_workspace_bytes(p->q, false, n_vec);
@@ -626,7 +629,8 @@ tq_status tq_decode_attention(const tq_params* kp, const tq_params* vp, const fl
                               const uint32_t* kcodes, const uint32_t* ksigns, const float* knorms,
                               const float* krnorms, const uint32_t* vcodes, const float* vnorms,
                               float* out, void* ws, size_t ws_bytes, void* stream) {
-  if (!kp || !vp || kp->mode != TQ_MODE_PROD || vp->mode != TQ_MODE_MSE) return TQ_ERR_INVALID_ARG;
+  if (!kp || !vp || kp->mode != TQ_MODE_PROD || (vp->mode != TQ_MODE_MSE && vp->mode != TQ_MODE_MSE_UNBIASED))
+    return TQ_ERR_INVALID_ARG;
   if (kp->q.d != vp->q.d || kp->q.rot != vp->q.rot) return TQ_ERR_INVALID_ARG;
   if (kp->q.rot != TQ_ROT_HADAMARD) return TQ_ERR_UNSUPPORTED;
   if (L < 1 || B < 1 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0) return TQ_ERR_INVALID_ARG;

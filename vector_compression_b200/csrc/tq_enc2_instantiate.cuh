@@ -36,6 +36,8 @@ cudaError_t enc2_by_mode(int mode, const QParams& qp, const SignMasks& sg, const
   switch (mode) {
     case MODE_MSE_ROW: return enc2_by_k<DP, T, MODE_MSE_ROW>(qp, sg, a, smem, ctas, st);
     case MODE_MSE_BLOCK: return enc2_by_k<DP, T, MODE_MSE_BLOCK>(qp, sg, a, smem, ctas, st);
+    case MODE_MSE_ROW_U: return enc2_by_k<DP, T, MODE_MSE_ROW_U>(qp, sg, a, smem, ctas, st);
+    case MODE_MSE_BLOCK_U: return enc2_by_k<DP, T, MODE_MSE_BLOCK_U>(qp, sg, a, smem, ctas, st);
     default: return enc2_by_k<DP, T, MODE_PROD>(qp, sg, a, smem, ctas, st);
   }
 }

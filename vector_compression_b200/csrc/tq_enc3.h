@@ -21,7 +21,8 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;      // 320
 constexpr uint32_t kTileBytes = kRows * kDP * 2;   // 32 KB of 16-bit input
 constexpr uint32_t kRotBytes = kDP * kDP * 2;      // 32 KB rotation operand
 
-enum { MODE_MSE_ROW = 0, MODE_MSE_BLOCK = 1, MODE_PROD = 2 };
+// *_U: Q_MSE with the unbiased (EDEN) scale n / <y, C[idx]> stored as the norm
+enum { MODE_MSE_ROW = 0, MODE_MSE_BLOCK = 1, MODE_PROD = 2, MODE_MSE_ROW_U = 3, MODE_MSE_BLOCK_U = 4 };
 
 // Division by a fixed d (1 <= d < 2^31) of n < 2^31 as a multiply and shift:
 // with s = ceil(log2 d) and M = floor(2^(32+s) / d) + 1 = 2^32 + mul, the

@@ -51,6 +51,8 @@ cudaError_t launch_f16(int mode, const CUtensorMap& map, const QParams& qp, cons
   switch (mode) {
     case MODE_MSE_ROW: return by_k<MODE_MSE_ROW>(map, qp, a, ctas, st);
     case MODE_MSE_BLOCK: return by_k<MODE_MSE_BLOCK>(map, qp, a, ctas, st);
+    case MODE_MSE_ROW_U: return by_k<MODE_MSE_ROW_U>(map, qp, a, ctas, st);
+    case MODE_MSE_BLOCK_U: return by_k<MODE_MSE_BLOCK_U>(map, qp, a, ctas, st);
     default: return by_k<MODE_PROD>(map, qp, a, ctas, st);
   }
 }

@@ -77,7 +77,10 @@ bool try_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_v
   a.norms = norms;
   a.rnorms = rnorms;
   a.err = err_word;
-  const int mode = prod ? MODE_PROD : (layout == TQ_LAYOUT_BLOCK32 ? MODE_MSE_BLOCK : MODE_MSE_ROW);
+  const bool blk = layout == TQ_LAYOUT_BLOCK32;
+  const int mode = prod ? MODE_PROD
+                        : qp.unbiased ? (blk ? MODE_MSE_BLOCK_U : MODE_MSE_ROW_U)
+                                      : (blk ? MODE_MSE_BLOCK : MODE_MSE_ROW);
   const int ctas = (int)std::min<int64_t>(a.n_tiles, (int64_t)num_sms);
   *err = dt == TQ_F16 ? launch_f16(mode, map, qp, a, ctas, st) : launch_bf16(mode, map, qp, a, ctas, st);
   return true;

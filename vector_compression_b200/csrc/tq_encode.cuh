@@ -138,7 +138,15 @@ __global__ void __launch_bounds__(128) encode_hadamard_kernel(
       uint32_t row_word = 0;
       quantize_pack<A>(v, idx, cb, k, lane, &row_word, blk, t, block_layout);
       if (!block_layout && lane < k * A) codes[slot * qp.code_words + lane] = row_word;
-      if (lane == 0) norms[slot] = n;
+      float nstore = n;
+      if (!PROD && qp.unbiased) {  // EDEN's scale n / <y, C[idx]>
+        float dot = 0.f;
+#pragma unroll
+        for (int a = 0; a < A; ++a) dot = fmaf(v[a], cb.c[idx[a]], dot);
+        dot = warp_sum(dot);
+        nstore = dot > 0.f ? n / dot : 0.f;
+      }
+      if (lane == 0) norms[slot] = nstore;
       if (PROD) {
         float rr = 0.f;
 #pragma unroll
@@ -194,12 +202,13 @@ __global__ void __launch_bounds__(128) normalize_rows_kernel(const T* __restrict
 }
 
 // Dense path, step 3: quantize rotated rows y (fp32 [nrows][d]) and pack.
-// Q_prod also overwrites y with r = y - C[idx] and writes rho.  One warp
-// per 32-vector task; the host splits chunks at segment and block boundaries.
+// Q_prod also overwrites y with r = y - C[idx] and writes rho; the unbiased
+// Q_MSE variant divides the stored norm by <y, C[idx]>.  One warp per
+// 32-vector task; the host splits chunks at segment and block boundaries.
 __global__ void __launch_bounds__(128) quantize_rows_kernel(
     QParams qp, float* __restrict__ y, int64_t seg_len, int64_t seg_cap, int64_t row0,
     int64_t nrows, int layout, bool prod, uint32_t* __restrict__ codes,
-    float* __restrict__ rnorms) {
+    float* __restrict__ norms, float* __restrict__ rnorms) {
   __shared__ SmemCodebook cb;
   load_codebook(cb, qp);
   __syncthreads();
@@ -223,15 +232,31 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(
       }
       for (int p = 0; p < k; ++p) dst[p * 32 * A + 32 * a + lane] = blk[p];
     }
+    if (qp.unbiased && !prod) {  // EDEN's scale n / <y, C[idx]> per row
+      for (int t = 0; t < nv; ++t) {
+        const float* yr = y + (first + t) * (int64_t)d;
+        float dot = 0.f;
+        for (int a = 0; a < A; ++a) {
+          const float v = yr[32 * a + lane];
+          dot = fmaf(v, cb.c[quantize_index(v, cb.b, nb)], dot);
+        }
+        dot = warp_sum(dot);
+        if (lane == 0) {
+          float* nr = norms + s * seg_cap + t0 + t;
+          *nr = dot > 0.f ? *nr / dot : 0.f;
+        }
+      }
+    }
     return;
   }
   for (int t = 0; t < nv; ++t) {
     float* yr = y + (first + t) * (int64_t)d;
     const int64_t slot = s * seg_cap + t0 + t;
-    float rr = 0.f;
+    float rr = 0.f, dot = 0.f;
     for (int a = 0; a < A; ++a) {
       const float v = yr[32 * a + lane];
       const int idx = quantize_index(v, cb.b, nb);
+      dot = fmaf(v, cb.c[idx], dot);
       for (int p = 0; p < k; ++p) {
         const uint32_t w = __ballot_sync(0xffffffffu, (idx >> p) & 1);
         if (lane == 0) codes[slot * qp.code_words + p * A + a] = w;
@@ -245,6 +270,9 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(
     if (prod) {
       rr = warp_sum(rr);
       if (lane == 0) rnorms[slot] = sqrtf(rr);
+    } else if (qp.unbiased) {  // EDEN's scale n / <y, C[idx]>
+      dot = warp_sum(dot);
+      if (lane == 0) norms[slot] = dot > 0.f ? norms[slot] / dot : 0.f;
     }
   }
 }

@@ -184,9 +184,10 @@ struct Thr {
 // thresholds; the planes of idx = s ? 2^(K-1) + mu : 2^(K-1) - 1 - mu are
 // then the top plane S and lower planes ~(S ^ M).  With RESID, v[i] is
 // replaced by the residual r = v * scale - C[idx] and rr accumulates r^2.
-template <int K, bool RESID>
+// With DOT, dot accumulates |v| |C[idx]| (= <v, C[idx]>, same signs).
+template <int K, bool RESID, bool DOT = false>
 __device__ __forceinline__ void quant32(float (&v)[32], const Thr<K>& th, const float (&cpos)[8],
-                                        float scale, uint32_t (&plane)[K], float& rr) {
+                                        float scale, uint32_t (&plane)[K], float& rr, float& dot) {
   uint32_t S = 0, M0 = 0, M1 = 0, M2 = 0;
 #pragma unroll
   for (int i = 31; i >= 0; --i) {
@@ -197,14 +198,14 @@ __device__ __forceinline__ void quant32(float (&v)[32], const Thr<K>& th, const 
     if (K == 2) {
       const bool m0 = a > th.t[0];
       M0 = (M0 << 1) | (m0 ? 1u : 0u);
-      if (RESID) cm = m0 ? cpos[1] : cpos[0];
+      if (RESID || DOT) cm = m0 ? cpos[1] : cpos[0];
     } else if (K == 3) {
       const bool m1 = a > th.t[1];
       const float t0 = m1 ? th.t[2] : th.t[0];
       const bool m0 = a > t0;
       M1 = (M1 << 1) | (m1 ? 1u : 0u);
       M0 = (M0 << 1) | (m0 ? 1u : 0u);
-      if (RESID) cm = m1 ? (m0 ? cpos[3] : cpos[2]) : (m0 ? cpos[1] : cpos[0]);
+      if (RESID || DOT) cm = m1 ? (m0 ? cpos[3] : cpos[2]) : (m0 ? cpos[1] : cpos[0]);
     } else if (K == 4) {
       const bool m2 = a > th.t[3];
       const float t1 = m2 ? th.t[5] : th.t[1];
@@ -214,7 +215,11 @@ __device__ __forceinline__ void quant32(float (&v)[32], const Thr<K>& th, const 
       M2 = (M2 << 1) | (m2 ? 1u : 0u);
       M1 = (M1 << 1) | (m1 ? 1u : 0u);
       M0 = (M0 << 1) | (m0 ? 1u : 0u);
+      if (DOT)
+        cm = m2 ? (m1 ? (m0 ? cpos[7] : cpos[6]) : (m0 ? cpos[5] : cpos[4]))
+                : (m1 ? (m0 ? cpos[3] : cpos[2]) : (m0 ? cpos[1] : cpos[0]));
     }
+    if (DOT) dot = fmaf(a, cm, dot);
     S = (S << 1) | (s ? 1u : 0u);
     if (RESID) {
       const float r = fmaf(y, scale, s ? -cm : cm);
@@ -340,7 +345,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
 
 // ------------------------------------------------------------------ kernel
 
-enum { MODE_MSE_ROW = 0, MODE_MSE_BLOCK = 1, MODE_PROD = 2 };
+// *_U: Q_MSE with the unbiased (EDEN) scale n / <y, C[idx]> stored as the norm
+enum { MODE_MSE_ROW = 0, MODE_MSE_BLOCK = 1, MODE_PROD = 2, MODE_MSE_ROW_U = 3, MODE_MSE_BLOCK_U = 4 };
 
 struct Args {
   Stage st;
@@ -361,6 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(QParams qp, SignMas
   __shared__ __align__(8) uint64_t mbar;
   __shared__ uint32_t tmem_base_s;
   constexpr bool PROD = MODE == MODE_PROD;
+  constexpr bool BLOCK = MODE == MODE_MSE_BLOCK || MODE == MODE_MSE_BLOCK_U;
+  constexpr bool UNB = MODE == MODE_MSE_ROW_U || MODE == MODE_MSE_BLOCK_U;
   constexpr int HALVES = DP / 128;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m = qp.m;
@@ -449,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(QParams qp, SignMas
     constexpr int ESZ = sizeof(T);
 
     // ---- per half (DP = 256: y_lo = H(x_lo + x_hi), y_hi = H(x_lo - x_hi))
-    float nrm2 = 0.f, rr2 = 0.f, scale = 0.f;
+    float nrm2 = 0.f, rr2 = 0.f, scale = 0.f, nrm = 0.f, dot = 0.f;
     Thr<K> th;
 #pragma unroll
     for (int i = 0; i < (int)(sizeof(th.t) / sizeof(float)); ++i) th.t[i] = 0.f;
@@ -488,9 +496,10 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(QParams qp, SignMas
         const float n = sqrtf(nrm2);
         const float sigma = n * sqrtf((float)DP);
         scale = n > 0.f ? qp.inv_sqrt_dpad / n : 0.f;
+        nrm = n;
 #pragma unroll
         for (int i = 0; i < (int)(sizeof(th.t) / sizeof(float)); ++i) th.t[i] = bpos[i] * sigma;
-        if (valid) a.norms[slot] = n;
+        if (!UNB && valid) a.norms[slot] = n;
       }
       fwht128(P);
 #pragma unroll
@@ -502,8 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(QParams qp, SignMas
           v[i] = j < 64 ? lo_of(P[j]) : hi_of(P[j - 64]);
         }
         uint32_t planes[K];
-        quant32<K, PROD>(v, th, cpos, scale, planes, rr2);
-        if (MODE == MODE_MSE_BLOCK) {
+        quant32<K, PROD, UNB>(v, th, cpos, scale, planes, rr2, dot);
+        if (BLOCK) {
           uint32_t* dst = a.codes + (s * (a.seg_cap / 32) + b) * (int64_t)(K * DP);
 #pragma unroll
           for (int p = 0; p < K; ++p) {
@@ -523,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(QParams qp, SignMas
           }
         }
       }
-      if (MODE != MODE_MSE_BLOCK && valid) {
+      if (!BLOCK && valid) {
         uint32_t* dst = a.codes + slot * (int64_t)(K * DP / 32);
 #pragma unroll
         for (int p = 0; p < K; ++p)
@@ -558,6 +567,10 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(QParams qp, SignMas
       }
     }
 
+    if (UNB && valid) {  // EDEN's scale n / <y, C[idx]>, with <y, C[idx]> = scale * dot
+      const float yc = dot * scale;
+      a.norms[slot] = yc > 0.f ? nrm / yc : 0.f;
+    }
     if (PROD) {
       const float rho = sqrtf(rr2);
       if (valid) a.rnorms[slot] = rho;

@@ -269,6 +269,21 @@ __device__ __forceinline__ void planes_from(uint32_t S, uint32_t M0, uint32_t M1
   if (K >= 4) plane[2] = ~(S ^ M2);
 }
 
+// |C[idx]| of one coordinate from a = |u| and the positive thresholds t,
+// taking the same decisions as quant32_mse (thermometer for K <= 3, binary
+// search for K = 4); cp = the positive centroids (unit domain).
+template <int K>
+__device__ __forceinline__ float mag_centroid(float a, const float (&t)[8], const float (&cp)[8]) {
+  if (K == 1) return cp[0];
+  if (K == 2) return a > t[0] ? cp[1] : cp[0];
+  if (K == 3) return a > t[1] ? (a > t[2] ? cp[3] : cp[2]) : (a > t[0] ? cp[1] : cp[0]);
+  const bool m2 = a > t[3];
+  const bool m1 = a > (m2 ? t[5] : t[1]);
+  const bool m0 = a > (m1 ? (m2 ? t[6] : t[2]) : (m2 ? t[4] : t[0]));
+  return m2 ? (m1 ? (m0 ? cp[7] : cp[6]) : (m0 ? cp[5] : cp[4]))
+            : (m1 ? (m0 ? cp[3] : cp[2]) : (m0 ? cp[1] : cp[0]));
+}
+
 // Q_MSE quantization of 32 coordinates u[0..32) (coordinate 32c + i in u[i])
 // against the positive thresholds t (boundaries times ||u||), bit planes
 // shifted into words (bit i = coordinate 32c + i).  K <= 3: every threshold
@@ -276,25 +291,54 @@ __device__ __forceinline__ void planes_from(uint32_t S, uint32_t M0, uint32_t M1
 // mu = T_0 + T_1 + T_2 has bits M1 = T_1 and M0 = T_0 ^ T_1 ^ T_2.  Each bit
 // costs one subtraction and one funnel shift.  K = 4: binary search of |u|
 // with integer masks.
-template <int K>
+// DOT (K <= 3): dot += sum |u| |C[idx]| from the thermometer, with cp the
+// positive centroids: |C| = cp_0 + sum_j T_j (cp_(j+1) - cp_j), and over the
+// 32 coordinates sum_{|u| > t_j} |u| = t_j popc(T_j) + sum max(|u| - t_j, 0),
+// where sum max(|u| - t, 0) = (sum |u| - 32 t + sum |t - |u||) / 2 needs one
+// addition per coordinate and threshold.  K = 4 selects |C| per coordinate.
+template <int K, bool DOT = false>
 __device__ __forceinline__ void quant32_mse(const uint32_t (&ur)[32], const float (&t)[8],
-                                            uint32_t (&plane)[K]) {
+                                            uint32_t (&plane)[K], const float (&cp)[8], float& dot) {
   uint32_t S = 0, M0 = 0, M1 = 0, M2 = 0;
   if (K <= 3) {
     uint32_t T0 = 0, T1 = 0, T2 = 0;
+    float sa = 0.f, D0 = 0.f, D1 = 0.f, D2 = 0.f;  // sum |u|, sum |t_j - |u||
 #pragma unroll
     for (int i = 31; i >= 0; --i) {
       const float u = __uint_as_float(ur[i]);
       const float a = fabsf(u);
       S = shift_in(S, sub_bits(0.0f, u));
-      if (K >= 2) T0 = shift_in(T0, sub_bits(t[0], a));
+      if (DOT) sa += a;
+      if (K >= 2) {
+        const uint32_t d0 = sub_bits(t[0], a);
+        T0 = shift_in(T0, d0);
+        if (DOT) D0 += fabsf(__uint_as_float(d0));
+      }
       if (K >= 3) {
-        T1 = shift_in(T1, sub_bits(t[1], a));
-        T2 = shift_in(T2, sub_bits(t[2], a));
+        const uint32_t d1 = sub_bits(t[1], a), d2 = sub_bits(t[2], a);
+        T1 = shift_in(T1, d1);
+        T2 = shift_in(T2, d2);
+        if (DOT) {
+          D1 += fabsf(__uint_as_float(d1));
+          D2 += fabsf(__uint_as_float(d2));
+        }
       }
     }
     M0 = K == 3 ? (T0 ^ T1 ^ T2) : T0;
     M1 = T1;
+    if (DOT) {
+      // sum over |u| > t of |u|
+      auto above = [&](float tj, uint32_t Tj, float Dj) {
+        return fmaf(tj, (float)__popc(Tj), 0.5f * (sa + fmaf(-32.0f, tj, Dj)));
+      };
+      float acc = cp[0] * sa;
+      if (K >= 2) acc = fmaf(cp[1] - cp[0], above(t[0], T0, D0), acc);
+      if (K >= 3) {
+        acc = fmaf(cp[2] - cp[1], above(t[1], T1, D1), acc);
+        acc = fmaf(cp[3] - cp[2], above(t[2], T2, D2), acc);
+      }
+      dot += acc;
+    }
   } else {
 #pragma unroll
     for (int i = 31; i >= 0; --i) {
@@ -308,6 +352,7 @@ __device__ __forceinline__ void quant32_mse(const uint32_t (&ur)[32], const floa
       M2 = M2 + M2 - m2;
       M1 = M1 + M1 - m1;
       M0 = M0 + M0 - m0;
+      if (DOT) dot = fmaf(a, mag_centroid<K>(a, t, cp), dot);
     }
   }
   planes_from<K>(S, M0, M1, M2, plane);
@@ -386,6 +431,8 @@ __device__ __forceinline__ uint32_t transpose32(uint32_t w, const TransposeCtl& 
 template <typename T, int K, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, QParams qp, Args a) {
+  constexpr bool BLOCK = MODE == MODE_MSE_BLOCK || MODE == MODE_MSE_BLOCK_U;
+  constexpr bool UNB = MODE == MODE_MSE_ROW_U || MODE == MODE_MSE_BLOCK_U;  // EDEN scale
   extern __shared__ unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages];
   __shared__ __align__(8) uint64_t bar_accf[2], bar_acce[2], bar_done;
@@ -505,9 +552,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t ubase = tmem + (uint32_t)grp * buf_cols + lane_off;
     const TransposeCtl tctl = make_transpose_ctl(lane);
     const int half_levels = 1 << (K - 1);
-    float bpos[8];
+    float bpos[8], cpos[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) bpos[i] = i < half_levels - 1 ? qp.boundaries[half_levels + i] : 0.f;
+    for (int i = 0; i < 8; ++i) {
+      bpos[i] = i < half_levels - 1 ? qp.boundaries[half_levels + i] : 0.f;
+      cpos[i] = UNB && i < half_levels ? qp.centroids[half_levels + i] : 0.f;
+    }
     for (int L = grp;; L += 2) {
       const int64_t tile = blockIdx.x + (int64_t)L * G;
       if (tile >= a.n_tiles) break;
@@ -523,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // BLOCK32: the warp's 32 rows are one block of one segment (segments hold
       // a multiple of 32 vectors and tiles start at multiples of 128 rows)
       uint32_t* blk = nullptr;
-      if (MODE == MODE_MSE_BLOCK) {
+      if (BLOCK) {
         const int64_t row0 = tile * kRows + quarter * 32;
         const int64_t seg0 = (int64_t)fastdiv((uint32_t)row0, a.seg_div);
         blk = a.codes + (seg0 * (a.seg_cap / 32) + (row0 - seg0 * a.seg_len) / 32) * (int64_t)(K * kDP);
@@ -556,8 +606,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       sumsq(rb);
       const float ssum = (ss0 + ss1) + (ss2 + ss3);       // ||u||^2 = d_pad ||x||^2
       const float nu = ssum > 0.f ? ssum * rsqrtf(ssum) : 0.f;
-      if (valid) a.norms[slot] = nu * qp.inv_sqrt_dpad;
+      if (!UNB && valid) a.norms[slot] = nu * qp.inv_sqrt_dpad;
       float th[8];
+      float dot = 0.f;  // UNB: sum |u| |C[idx]| = nu <y, C[idx]>
 #pragma unroll
       for (int i = 0; i < 8; ++i) th[i] = bpos[i] * nu;
       uint32_t rowq[K][4];
@@ -565,8 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // quantize chunk c (coordinates 32c .. 32c+31) held in r
       auto process = [&](const int c, const uint32_t (&r)[32]) {
         uint32_t planes[K];
-        quant32_mse<K>(r, th, planes);
-        if (MODE == MODE_MSE_BLOCK) {
+        quant32_mse<K, UNB>(r, th, planes, cpos, dot);
+        if (BLOCK) {
 #pragma unroll
           for (int p = 0; p < K; ++p) {
             const uint32_t word = transpose32(valid ? planes[p] : 0u, tctl);
@@ -591,7 +642,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bar_acce[grp]));
       process(1, rb);
-      if (MODE != MODE_MSE_BLOCK && valid) {
+      // EDEN: n / <y, C[idx]> = (nu / sqrt(d_pad)) nu / dot
+      if (UNB && valid) a.norms[slot] = dot > 0.f ? nu * qp.inv_sqrt_dpad * nu / dot : 0.f;
+      if (!BLOCK && valid) {
         uint4* dst = reinterpret_cast<uint4*>(a.codes + slot * (int64_t)(K * 4));
 #pragma unroll
         for (int p = 0; p < K; ++p) dst[p] = make_uint4(rowq[p][0], rowq[p][1], rowq[p][2], rowq[p][3]);

@@ -21,6 +21,7 @@ struct QParams {
   int rot;        // tq_rot
   int code_words; // k * ceil(d_pad / 32): ROW words per vector
   int sign_words; // m / 32
+  int unbiased;   // Q_MSE with the unbiased (EDEN) per-vector scale in place of the norm
   float inv_sqrt_dpad;
   float kappa;    // sqrt(pi/2) / m
   float centroids[kMaxLevels];

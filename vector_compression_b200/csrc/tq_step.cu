@@ -75,7 +75,8 @@ extern "C" tq_status tq_decode_step(const tq_params* kp, const tq_params* vp, co
                                     uint32_t* kcodes, uint32_t* ksigns, float* knorms, float* krnorms,
                                     uint32_t* vcodes, float* vnorms, float* out, void* ws,
                                     size_t ws_bytes, void* stream) {
-  if (!kp || !vp || kp->mode != TQ_MODE_PROD || vp->mode != TQ_MODE_MSE) return TQ_ERR_INVALID_ARG;
+  if (!kp || !vp || kp->mode != TQ_MODE_PROD || (vp->mode != TQ_MODE_MSE && vp->mode != TQ_MODE_MSE_UNBIASED))
+    return TQ_ERR_INVALID_ARG;
   if (kp->q.d != vp->q.d || kp->q.rot != vp->q.rot) return TQ_ERR_INVALID_ARG;
   if (kp->q.rot != TQ_ROT_HADAMARD) return TQ_ERR_UNSUPPORTED;
   if (dt != TQ_F32 && dt != TQ_F16 && dt != TQ_BF16) return TQ_ERR_INVALID_ARG;
