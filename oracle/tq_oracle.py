@@ -39,6 +39,8 @@ DESIGN.md):
 * QJL scale sqrt(pi/2)/m with m rows of S ([EXPL] §8 has m = d).
 * The residual and S act in the rotated domain ([EXPL] §8: r = Pi x - y_mse).
 * A zero vector has norm 0 and is encoded from the zero rotated vector.
+* fp16 residual norms (storage variant): rho rounded to the nearest IEEE
+  binary16 value, ties to even.
 * Unbiased per-vector scale (EDEN; DRIVE at one bit): the Q_MSE codes are
   kept and the stored scale is S = ||x||^2 / <Pi x, C[idx]> = n / <y, C[idx]>
   in place of n, so that the unchanged decoder n Pi^T C[idx] becomes
@@ -369,12 +371,16 @@ class Quantizer:
     definition of Q_prod).
     """
 
-    def __init__(self, d: int, bits: int, *, prod: bool, draws: dict, unbiased: bool = False):
+    def __init__(self, d: int, bits: int, *, prod: bool, draws: dict, unbiased: bool = False,
+                 rnorm_f16: bool = False):
         self.d = d
         self.bits = bits
         self.prod = prod
         # Q_MSE with EDEN's unbiased per-vector scale in place of the norm
         self.unbiased = bool(unbiased) and not prod
+        # Q_prod storage variant: residual norms kept as IEEE fp16 ([PYT]
+        # Pattern 4 memory formula, one float16 residual norm per key)
+        self.rnorm_f16 = bool(rnorm_f16) and prod
         self.k = bits - 1 if prod else bits
         if draws.get("G") is not None:
             self.rot = Rotation(d, G=draws["G"])
@@ -426,7 +432,8 @@ class Quantizer:
             rho = np.sqrt(np.sum(r * r, axis=-1))
             z = r @ self.S.T
             sig = (z >= 0).astype(np.int64)
-            out.update(rnorms=rho.astype(np.float32), signs=pack_signs(sig), z=z, rho64=rho)
+            out.update(rnorms=rho.astype(np.float16 if self.rnorm_f16 else np.float32),
+                       signs=pack_signs(sig), z=z, rho64=rho)
         return out
 
     def unbiased_scale(self, n, y, idx):

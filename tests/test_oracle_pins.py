@@ -405,6 +405,45 @@ def test_unbiased_scale_over_haar_rotations():
     assert np.any(np.abs(lam * x - x) > 8 * se)  # the test separates the biased decoder
 
 
+def _fp16_round_reference(v):
+    """Nearest IEEE binary16 value of positive doubles, ties to even, from the
+    format's definition (11 significant bits; exponents -14..15; below 2^-14
+    a fixed step of 2^-24), independent of numpy's float16 cast."""
+    out = []
+    for x in v:
+        x = float(x)
+        if x == 0.0:
+            out.append(0.0)
+            continue
+        e = max(math.floor(math.log2(x)), -14)
+        step = 2.0 ** (e - 10)
+        q, r = divmod(x, step)
+        if r > step / 2 or (r == step / 2 and int(q) % 2 == 1):
+            q += 1
+        out.append(q * step)
+    return np.array(out)
+
+
+def test_fp16_residual_norms_round_to_nearest_even():
+    # storage variant: rho kept as binary16; checked against the format's
+    # definition, including exact ties and subnormal residual norms
+    d, bits = 128, 3
+    q16 = o.Quantizer(d, bits, prod=True, draws=_draws(d, 64, 5), rnorm_f16=True)
+    x = np.random.default_rng(71).standard_normal((300, d)) * 7.0
+    e = q16.encode(x)
+    assert e["rnorms"].dtype == np.float16
+    np.testing.assert_array_equal(e["rnorms"].astype(np.float64), _fp16_round_reference(e["rho64"]))
+    rel = np.abs(e["rnorms"].astype(np.float64) / e["rho64"] - 1.0)
+    assert rel.max() <= 2.0 ** -11
+    ties = np.array([1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 0.5 + 2.0 ** -12, 3.0 * 2.0 ** -25])
+    np.testing.assert_array_equal(ties.astype(np.float16).astype(np.float64), _fp16_round_reference(ties))
+    # codes, signs and norms are those of the fp32 variant
+    q32 = o.Quantizer(d, bits, prod=True, draws=_draws(d, 64, 5))
+    e32 = q32.encode(x)
+    for k in ("codes", "signs", "norms"):
+        assert np.array_equal(e[k], e32[k])
+
+
 def test_residual_norm_expectation():
     # Residual energy: E||r||^2 = d_pad * C(f, b-1) over random unit inputs
     # (the notes' E||r|| = sqrt(C) read as the second moment); dense Haar
