@@ -65,6 +65,12 @@ typedef enum { TQ_F32 = 0, TQ_F16 = 1, TQ_BF16 = 2 } tq_dtype;
 typedef enum { TQ_ROT_HADAMARD = 0, TQ_ROT_DENSE = 1 } tq_rot;
 typedef enum { TQ_MODE_MSE = 0, TQ_MODE_PROD = 1, TQ_MODE_MSE_UNBIASED = 2 } tq_mode;
 typedef enum { TQ_LAYOUT_ROW = 0, TQ_LAYOUT_BLOCK32 = 1 } tq_layout;
+/* Storage flag OR'ed into the mode of tq_params_create (TQ_MODE_PROD only):
+ * residual norms rho are stored as IEEE fp16 (round to nearest even), as in
+ * [PYT] Pattern 4's memory formula ("1 float16 per vector").  Every rnorms /
+ * krnorms argument of such a handle then points to uint16_t storage with
+ * the same element count (pass the address cast to float*). */
+typedef enum { TQ_STORE_RNORM_F16 = 0x100 } tq_store_flag;
 
 typedef struct tq_params tq_params; /* opaque quantizer description */
 
@@ -117,6 +123,8 @@ tq_status tq_make_rotation(int d, const double* G, float* Pi);
  *           S Pi^T C[idx], whose component along x is exactly x and whose
  *           mean over uniformly random rotations is x.  Accepted wherever
  *           TQ_MODE_MSE is.
+ *           TQ_MODE_PROD | TQ_STORE_RNORM_F16 stores the residual norms in
+ *           fp16 (see tq_store_flag).
  *   rot     TQ_ROT_HADAMARD: Pi = H D / sqrt(d_pad), d_pad = next power of
  *           two >= d (at least 32), the vector zero-padded ([EXPL] §0.9,
  *           [FVQ]); d_pad must be 32..256.

@@ -15,7 +15,7 @@ import numpy as np
 
 from . import _lib as L
 from ._lib import (BF16, F16, F32, LAYOUT_BLOCK32, LAYOUT_ROW, MODE_MSE, MODE_MSE_UNBIASED, MODE_PROD,  # noqa: F401
-                   ROT_DENSE, ROT_HADAMARD, TQError)
+                   ROT_DENSE, ROT_HADAMARD, STORE_RNORM_F16, TQError)
 
 __all__ = [
     "TQParams", "tq_build_codebook", "tq_make_rotation", "tq_params_create", "tq_encode_mse", "tq_encode_prod",
@@ -98,7 +98,9 @@ class TQParams:
             C.byref(self._h)))
         vals = [C.c_int() for _ in range(5)]
         L.check("tq_params_info", L.lib().tq_params_info(self._h, *[C.byref(v) for v in vals]))
-        self.d, self.bits, self.mode, self.rot = d, bits, mode, rot
+        self.d, self.bits, self.mode, self.rot = d, bits, mode & 0xFF, rot
+        # residual norms stored as fp16 (torch.float16 tensors) instead of fp32
+        self.rnorm_dtype = "float16" if mode & STORE_RNORM_F16 else "float32"
         self.d_pad, self.k, self.code_words, self.sign_words, self.m = [v.value for v in vals]
 
     @property
@@ -185,7 +187,7 @@ def tq_encode_prod(p: TQParams, x, seg_len: int = 0, seg_cap: int = 0, out=None,
         out = (torch.zeros((ns * sc, p.code_words), dtype=torch.int32, device=dev),
                torch.zeros((ns * sc, p.sign_words), dtype=torch.int32, device=dev),
                torch.zeros(ns * sc, dtype=torch.float32, device=dev),
-               torch.zeros(ns * sc, dtype=torch.float32, device=dev))
+               torch.zeros(ns * sc, dtype=getattr(torch, p.rnorm_dtype), device=dev))
     codes, signs, norms, rnorms = out
     need = C.c_size_t()
     L.check("tq_encode_workspace_size", L.lib().tq_encode_workspace_size(p.handle, n, C.byref(need)))

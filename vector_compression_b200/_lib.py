@@ -17,6 +17,7 @@ STATUS = {
 F32, F16, BF16 = 0, 1, 2
 ROT_HADAMARD, ROT_DENSE = 0, 1
 MODE_MSE, MODE_PROD, MODE_MSE_UNBIASED = 0, 1, 2
+STORE_RNORM_F16 = 0x100  # OR'ed into MODE_PROD: residual norms stored as fp16
 LAYOUT_ROW, LAYOUT_BLOCK32 = 0, 1
 
 # exported symbol -> (restype, argtypes)

@@ -411,6 +411,7 @@ int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q
     p2.ksigns = ksigns;
     p2.knorms = knorms;
     p2.krnorms = krnorms;
+    p2.kr16 = kp.rnorm_f16;
     p2.vcodes = vcodes;
     p2.vnorms = vnorms;
     p2.part = part;

@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kAttnThreads) attention_chunk_kernel(
         }
       }
       kn = knorms[kbase + t];
-      kr = kp.kappa * krnorms[kbase + t];
+      kr = kp.kappa * get_rnorm(krnorms, kbase + t, kp.rnorm_f16);
     }
     const float vn = valid ? vnorms[kbase + t] : 0.f;
 #pragma unroll

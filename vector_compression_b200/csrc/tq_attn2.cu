@@ -223,8 +223,8 @@ __global__ void __launch_bounds__(kThreads) attn_chunk_kernel(Params P) {
       }
     }
     const float n1 = ok1 ? P.knorms[krow0 + T1] : 0.f, n2 = ok2 ? P.knorms[krow0 + T2] : 0.f;
-    const float kr1 = ok1 ? kappa * P.krnorms[krow0 + T1] : 0.f;
-    const float kr2 = ok2 ? kappa * P.krnorms[krow0 + T2] : 0.f;
+    const float kr1 = ok1 ? kappa * get_rnorm(P.krnorms, krow0 + T1, P.kr16) : 0.f;
+    const float kr2 = ok2 ? kappa * get_rnorm(P.krnorms, krow0 + T2, P.kr16) : 0.f;
     const float vn1 = ok1 ? P.vnorms[krow0 + T1] : 0.f, vn2 = ok2 ? P.vnorms[krow0 + T2] : 0.f;
 
     float am[4] = {0.f, 0.f, 0.f, 0.f}, aq[4] = {0.f, 0.f, 0.f, 0.f};

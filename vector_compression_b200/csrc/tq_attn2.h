@@ -19,7 +19,8 @@ struct Params {
   const uint32_t* kcodes;
   const uint32_t* ksigns;
   const float* knorms;
-  const float* krnorms;
+  const float* krnorms;  // fp32, or fp16 storage when kr16
+  int kr16;
   const uint32_t* vcodes;
   const float* vnorms;
   float* part;

@@ -213,11 +213,13 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
   // round_up(n, 4) tokens (inside the cache: cap >= round_up(seq, 32))
   auto issue_keys = [&](int64_t s) {
     const uint32_t n4 = (uint32_t)((min64(SC, t_end - s) + 3) & ~3);
-    mbar_expect(bk, n4 * (KW * 4 + SW * 4 + 8));
+    // fp16 residual norms: 8-token granules keep the copy a multiple of 16 bytes
+    const uint32_t kr_bytes = P.kr16 ? ((n4 + 7) & ~7u) * 2 : n4 * 4;
+    mbar_expect(bk, n4 * (KW * 4 + SW * 4 + 4) + kr_bytes);
     bulk_g2s(s_kc, P.kcodes + (krow0 + s) * KW, n4 * KW * 4, bk);
     bulk_g2s(s_ks, P.ksigns + (krow0 + s) * SW, n4 * SW * 4, bk);
     bulk_g2s(s_kn, P.knorms + krow0 + s, n4 * 4, bk);
-    bulk_g2s(s_kr, P.krnorms + krow0 + s, n4 * 4, bk);
+    bulk_g2s(s_kr, reinterpret_cast<const char*>(P.krnorms) + (krow0 + s) * (P.kr16 ? 2 : 4), kr_bytes, bk);
   };
   // values of the sub-chunk at s: its 32-token blocks and the value norms
   auto issue_values = [&](int64_t s) {
@@ -347,7 +349,8 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
         k2[KW] = b.x; k2[KW + 1] = b.y;
       }
       const float n1 = s_kn[R1], n2 = s_kn[R2];
-      const float r1 = s_kr[R1], r2 = s_kr[R2];
+      const float r1 = P.kr16 ? __half2float(reinterpret_cast<const __half*>(s_kr)[R1]) : s_kr[R1];
+      const float r2 = P.kr16 ? __half2float(reinterpret_cast<const __half*>(s_kr)[R2]) : s_kr[R2];
       int acc[FK + 1][NT + 1][4];
 #pragma unroll
       for (int f = 0; f <= FK; ++f)

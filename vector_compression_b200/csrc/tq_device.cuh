@@ -22,6 +22,15 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
   return __bfloat162float(v);
 }
 
+// Residual norms: fp32, or fp16 storage behind the same pointer (QParams::rnorm_f16).
+__device__ __forceinline__ void put_rnorm(float* p, int64_t i, float v, int f16) {
+  if (f16) reinterpret_cast<__half*>(p)[i] = __float2half_rn(v);
+  else p[i] = v;
+}
+__device__ __forceinline__ float get_rnorm(const float* p, int64_t i, int f16) {
+  return f16 ? __half2float(reinterpret_cast<const __half*>(p)[i]) : p[i];
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

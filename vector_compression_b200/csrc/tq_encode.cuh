@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(128) encode_hadamard_kernel(
         rr = warp_sum(rr);
         __syncwarp();
         qjl_signs(qp, r_s[wib], lane, signs + slot * qp.sign_words);
-        if (lane == 0) rnorms[slot] = sqrtf(rr);
+        if (lane == 0) put_rnorm(rnorms, slot, sqrtf(rr), qp.rnorm_f16);
         __syncwarp();
       }
     }
@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(
     }
     if (prod) {
       rr = warp_sum(rr);
-      if (lane == 0) rnorms[slot] = sqrtf(rr);
+      if (lane == 0) put_rnorm(rnorms, slot, sqrtf(rr), qp.rnorm_f16);
     } else if (qp.unbiased) {  // EDEN's scale n / <y, C[idx]>
       dot = warp_sum(dot);
       if (lane == 0) norms[slot] = dot > 0.f ? norms[slot] / dot : 0.f;

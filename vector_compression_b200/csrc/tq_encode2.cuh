@@ -573,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(QParams qp, SignMas
     }
     if (PROD) {
       const float rho = sqrtf(rr2);
-      if (valid) a.rnorms[slot] = rho;
+      if (valid) put_rnorm(a.rnorms, slot, rho, qp.rnorm_f16);
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
       __syncthreads();

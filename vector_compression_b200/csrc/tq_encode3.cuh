@@ -876,7 +876,7 @@ __global__ void __launch_bounds__(prod_threads<TPR>(), 1)
       if (cg == 0 && valid_p) {
         const float4 q = *reinterpret_cast<const float4*>(&rr_part[Lp & 1][rloc][0]);
         const float t = TPR == 4 ? (q.x + q.y) + (q.z + q.w) : q.x + q.y;
-        a.rnorms[slot_p] = t > 0.f ? t * rsqrtf(t) * (1.0f / 1024.0f) : 0.f;
+        put_rnorm(a.rnorms, slot_p, t > 0.f ? t * rsqrtf(t) * (1.0f / 1024.0f) : 0.f, qp.rnorm_f16);
       }
     };
 

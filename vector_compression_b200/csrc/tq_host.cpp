@@ -289,7 +289,11 @@ tq_status tq_params_create(int d, int bits, tq_mode mode, tq_rot rot, int m, con
   if (!out) return TQ_ERR_INVALID_ARG;
   *out = nullptr;
   if (d < 1 || d > tq::kMaxDim) return TQ_ERR_INVALID_ARG;
+  const int store_flags = (int)mode & ~0xFF;
+  mode = (tq_mode)((int)mode & 0xFF);
   if (mode != TQ_MODE_MSE && mode != TQ_MODE_PROD && mode != TQ_MODE_MSE_UNBIASED) return TQ_ERR_INVALID_ARG;
+  if (store_flags & ~(int)TQ_STORE_RNORM_F16) return TQ_ERR_INVALID_ARG;
+  if ((store_flags & TQ_STORE_RNORM_F16) && mode != TQ_MODE_PROD) return TQ_ERR_INVALID_ARG;
   if (rot != TQ_ROT_HADAMARD && rot != TQ_ROT_DENSE) return TQ_ERR_INVALID_ARG;
   const bool prod = mode == TQ_MODE_PROD;
   if (!prod && (bits < 1 || bits > 4)) return TQ_ERR_INVALID_ARG;
@@ -324,6 +328,7 @@ tq_status tq_params_create(int d, int bits, tq_mode mode, tq_rot rot, int m, con
   q.m = m;
   q.rot = rot;
   q.unbiased = mode == TQ_MODE_MSE_UNBIASED ? 1 : 0;
+  q.rnorm_f16 = (store_flags & TQ_STORE_RNORM_F16) ? 1 : 0;
   q.code_words = k * ((d_pad + 31) / 32);
   q.sign_words = m / 32;
   q.inv_sqrt_dpad = (float)(1.0 / std::sqrt((double)d_pad));

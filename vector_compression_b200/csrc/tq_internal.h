@@ -22,6 +22,7 @@ struct QParams {
   int code_words; // k * ceil(d_pad / 32): ROW words per vector
   int sign_words; // m / 32
   int unbiased;   // Q_MSE with the unbiased (EDEN) per-vector scale in place of the norm
+  int rnorm_f16;  // residual norms stored as fp16 (uint16 storage behind the float* arguments)
   float inv_sqrt_dpad;
   float kappa;    // sqrt(pi/2) / m
   float centroids[kMaxLevels];

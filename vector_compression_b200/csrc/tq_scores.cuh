@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kScoreThreads) scores_kernel(
     }
   }
   const float n = norms[t];
-  const float kr = m > 0 ? qp.kappa * rnorms[t] : 0.f;
+  const float kr = m > 0 ? qp.kappa * get_rnorm(rnorms, t, qp.rnorm_f16) : 0.f;
 #pragma unroll
   for (int a = 0; a < kMaxQT; ++a)
     if (a < nql) scores[(q0 + a) * n_vec + t] = n * (am[a] + kr * aq[a]);
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(128) decode_hadamard_kernel(
     v[a] = cb.c[idx];
   }
   if (signs && qp.m > 0) {
-    const float kr = qp.kappa * rnorms[slot];
+    const float kr = qp.kappa * get_rnorm(rnorms, slot, qp.rnorm_f16);
     const uint32_t* sw = signs + slot * qp.sign_words;
 #pragma unroll
     for (int a = 0; a < A; ++a) {
@@ -305,7 +305,7 @@ __global__ void __launch_bounds__(128) decode_dense_kernel(
         const float sg = ((sw[i / 32] >> (i % 32)) & 1u) ? 1.f : -1.f;
         acc = fmaf(__ldg(qp.S + (size_t)i * d + j), sg, acc);
       }
-      v = fmaf(qp.kappa * rnorms[slot], acc, v);
+      v = fmaf(qp.kappa * get_rnorm(rnorms, slot, qp.rnorm_f16), acc, v);
     }
     ys[32 * a + lane] = v;
   }

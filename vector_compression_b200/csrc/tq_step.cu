@@ -100,7 +100,9 @@ extern "C" tq_status tq_decode_step(const tq_params* kp, const tq_params* vp, co
   // keys: segment g of one vector -> slot g * cap, shifted by pos slots
   int e = tq::launch_encode(kp->q, true, k_new, dt, n, d, 1, cap, TQ_LAYOUT_ROW,
                             kcodes + pos * kp->q.code_words, ksigns + pos * kp->q.sign_words, knorms + pos,
-                            krnorms + pos, nullptr, stream);
+                            // fp16 residual norms are 2-byte slots
+                            reinterpret_cast<float*>(reinterpret_cast<char*>(krnorms) + pos * (kp->q.rnorm_f16 ? 2 : 4)),
+                            nullptr, stream);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
   // values: ROW codes into the workspace, then into bit pos % 32 of their blocks
   e = tq::launch_encode(vp->q, false, v_new, dt, n, d, 1, 1, TQ_LAYOUT_ROW, tmp, nullptr, tmp_norms, nullptr,
