@@ -89,6 +89,8 @@ def test_params_validation():
     S = np.full((128, 128), 0.1, np.float32)  # not fp16-representable
     assert lib.tq_params_create(128, 3, 1, 0, 128, p, S.ctypes.data_as(C.c_void_p), None, C.byref(h)) == 1
     assert lib.tq_params_create(128, 3, 3, 0, 0, p, None, None, C.byref(h)) == 1    # no mode 3
+    assert lib.tq_params_create(128, 3, 0x100, 0, 0, p, None, None, C.byref(h)) == 1  # fp16 rho needs PROD
+    assert lib.tq_params_create(128, 3, 0x201, 0, 128, p, None, None, C.byref(h)) == 1  # unknown flag
 
 
 def test_unbiased_mode_handle():
