@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--cpu-sample-groups", type=int, default=6)
     ap.add_argument("--value-scale", default="norm", choices=["norm", "unbiased"],
                     help="per-vector scale stored with the values: the norm, or EDEN's unbiased scale")
+    ap.add_argument("--rnorm-f16", action="store_true", help="store the keys' residual norms as fp16")
     ap.add_argument("--qjl-rows", type=int, default=0,
                     help="QJL projection rows m of the keys (0 = the padded head dim; d_pad / 2 is the half-size variant)")
     return ap.parse_args()
@@ -62,11 +63,11 @@ def peaks():
     return 6650.0, "fallback"
 
 
-def workload_bytes(cfg, k_words, k_signs, v_words):
+def workload_bytes(cfg, k_words, k_signs, v_words, rnorm_bytes=4):
     """Algorithmic bytes of one step, split per kernel family."""
     n = cfg.layers * cfg.batch * cfg.kv_heads * cfg.seq
     esz = 2 if cfg.dtype in ("float16", "bfloat16") else 4
-    key_row = 4 * (k_words + k_signs) + 8   # codes + signs + norm + residual norm
+    key_row = 4 * (k_words + k_signs) + 4 + rnorm_bytes   # codes + signs + norm + residual norm
     val_row = 4 * v_words + 4               # codes + norm
     nq = cfg.layers * cfg.batch * cfg.q_heads
     return {
@@ -143,7 +144,8 @@ class OracleSample:
     (layer, batch, kv-head) groups of one layer, each fully encoded (keys
     Q_prod, values Q_MSE) and attended by its G query heads."""
 
-    def __init__(self, cfg, groups: int, layer: int = 0, m: int = 0, unbiased: bool = False):
+    def __init__(self, cfg, groups: int, layer: int = 0, m: int = 0, unbiased: bool = False,
+                 rnorm_f16: bool = False):
         import torch
 
         from oracle import tq_oracle as o
@@ -154,7 +156,7 @@ class OracleSample:
         self.cores = torch.get_num_threads()
         kd = synth.method_draws(cfg.head_dim, m or cfg.d_pad, cfg.seed, stream=1)
         vd = synth.method_draws(cfg.head_dim, cfg.d_pad, cfg.seed, stream=2)
-        self.kq = o.Quantizer(cfg.head_dim, cfg.key_bits, prod=True, draws=kd)
+        self.kq = o.Quantizer(cfg.head_dim, cfg.key_bits, prod=True, draws=kd, rnorm_f16=rnorm_f16)
         self.vq = o.Quantizer(cfg.head_dim, cfg.value_bits, prod=False, draws=vd, unbiased=unbiased)
         one = cfg.scaled(layers=1)
         K, V = synth.kv_cache(one, device="cpu", layers=range(layer, layer + 1))
@@ -164,7 +166,8 @@ class OracleSample:
         self.V = V.float().numpy().astype(np.float64).reshape(-1, cfg.seq, cfg.head_dim)[: self.groups]
         self.q = q.numpy().astype(np.float64).reshape(-1, cfg.group, cfg.head_dim)[: self.groups]
         nb = workload_bytes(cfg.scaled(layers=1, batch=1, kv_heads=1, q_heads=cfg.group),
-                            self.kq.k * self.kq.d_pad // 32, self.kq.m // 32, self.vq.k * self.vq.d_pad // 32)
+                            self.kq.k * self.kq.d_pad // 32, self.kq.m // 32, self.vq.k * self.vq.d_pad // 32,
+                            rnorm_bytes=2 if rnorm_f16 else 4)
         self.bytes = (nb["encode_prod"] + nb["encode_mse"] + nb["attention"]) * self.groups
         self.sample = f"{self.groups} (layer, batch, kv-head) groups x {cfg.seq} tokens of layer {layer}"
 
@@ -186,7 +189,7 @@ def run_reference(args, cfg):
     if rank != 0:
         return
     sample = OracleSample(cfg, max(1, args.cpu_sample_groups // 3), m=args.qjl_rows,
-                          unbiased=args.value_scale == "unbiased")
+                          unbiased=args.value_scale == "unbiased", rnorm_f16=args.rnorm_f16)
     for _ in range(args.warmup):
         sample.run()
     vals, secs = [], []
@@ -235,7 +238,8 @@ def main():
     m = args.qjl_rows or cfg.d_pad
     kd = synth.method_draws(cfg.head_dim, m, cfg.seed, stream=1)
     vd = synth.method_draws(cfg.head_dim, cfg.d_pad, cfg.seed, stream=2)
-    kp = tq.TQParams(cfg.head_dim, cfg.key_bits, tq.MODE_PROD, tq.ROT_HADAMARD, m=m,
+    kmode = tq.MODE_PROD | (tq.STORE_RNORM_F16 if args.rnorm_f16 else 0)
+    kp = tq.TQParams(cfg.head_dim, cfg.key_bits, kmode, tq.ROT_HADAMARD, m=m,
                      signs=kd["signs"], S=kd["S"])
     vmode = tq.MODE_MSE_UNBIASED if args.value_scale == "unbiased" else tq.MODE_MSE
     vp = tq.TQParams(cfg.head_dim, cfg.value_bits, vmode, tq.ROT_HADAMARD, signs=vd["signs"])
@@ -245,7 +249,8 @@ def main():
     n = cfg.layers * cfg.batch * cfg.kv_heads * seq
     kc = (torch.empty((n, kp.code_words), dtype=torch.int32, device=dev),
           torch.empty((n, kp.sign_words), dtype=torch.int32, device=dev),
-          torch.empty(n, dtype=torch.float32, device=dev), torch.empty(n, dtype=torch.float32, device=dev))
+          torch.empty(n, dtype=torch.float32, device=dev),
+          torch.empty(n, dtype=getattr(torch, kp.rnorm_dtype), device=dev))
     vcodes = torch.empty((n // 32, vp.k * vp.d_pad), dtype=torch.int32, device=dev)
     vnorms = torch.empty(n, dtype=torch.float32, device=dev)
     out = torch.empty((cfg.layers, cfg.batch, cfg.q_heads, cfg.head_dim), dtype=torch.float32, device=dev)
@@ -253,7 +258,8 @@ def main():
                                                            cfg.kv_heads, seq), dtype=torch.uint8, device=dev)
     scale = synth.softmax_scale(cfg.head_dim)
     stream = torch.cuda.current_stream()
-    nb = workload_bytes(cfg, kp.code_words, kp.sign_words, vp.k * vp.d_pad // 32)
+    nb = workload_bytes(cfg, kp.code_words, kp.sign_words, vp.k * vp.d_pad // 32,
+                        rnorm_bytes=2 if args.rnorm_f16 else 4)
 
     ev = {k: [] for k in ("encode_prod", "encode_mse", "attention")}
 
@@ -338,7 +344,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1:
-        s = OracleSample(cfg, args.cpu_sample_groups, m=args.qjl_rows, unbiased=args.value_scale == "unbiased")
+        s = OracleSample(cfg, args.cpu_sample_groups, m=args.qjl_rows, unbiased=args.value_scale == "unbiased",
+                         rnorm_f16=args.rnorm_f16)
         v, dt = s.run()
         cpu = {"value": v, "unit": UNIT, "cores": s.cores, "kind": "oracle", "sample": s.sample, "seconds": dt}
 
@@ -350,6 +357,7 @@ def main():
             "config": {"workload": cfg.name, "layers": cfg.layers, "batch": cfg.batch, "kv_heads": cfg.kv_heads,
                        "q_heads": cfg.q_heads, "head_dim": cfg.head_dim, "seq": cfg.seq, "input_dtype": cfg.dtype,
                        "key_bits": cfg.key_bits, "value_bits": cfg.value_bits, "qjl_m": kp.m, "value_scale": args.value_scale,
+                       "rnorm_dtype": kp.rnorm_dtype,
                        "rotation": "randomized Hadamard", "l2": "inputs larger than L2 (no flush)",
                        "bytes_per_step": step_bytes, "parallelism": f"replica x{world}"},
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["GB/s"], "peak": peak,
