@@ -184,6 +184,25 @@ class OracleSample:
         return self.bytes / dt / 1e9, dt
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks (every rank calls this at the same
+    point; a single process returns its own)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(step_bytes: int, world: int, ms: float) -> float:
+    """Whole-job GB/s: every rank processes step_bytes per step (weak scaling),
+    timed by the slowest rank's ms per step."""
+    return world * step_bytes / (ms * 1e-3) / 1e9
+
+
 def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -302,16 +321,12 @@ def main():
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    ms = t_start.elapsed_time(t_end) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, dev)
     tq.tq_sync_check()
 
     kern_ms = {k: statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in ev.items()}
     step_bytes = nb["encode_prod"] + nb["encode_mse"] + nb["attention"]
-    value = world * step_bytes / (ms * 1e-3) / 1e9
+    value = job_throughput(step_bytes, world, ms)
     peak, peak_kind = peaks()
     kernels = {}
     for k in ("encode_prod", "encode_mse", "attention"):
@@ -335,12 +350,10 @@ def main():
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, tq, kp, vp, K, V, q, kc, vcodes, vnorms, out, ws, seq, cap, scale, step_bytes)
-    if world > 1:
-        t = torch.tensor([e2e["ms"] if e2e else 0.0], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        if e2e:
-            e2e["ms"] = float(t.item())
-            e2e["value"] = world * step_bytes / (e2e["ms"] * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(e2e["ms"] if e2e else 0.0, dev)
+    if e2e:
+        e2e["ms"] = e2e_ms
+        e2e["value"] = job_throughput(step_bytes, world, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1:
