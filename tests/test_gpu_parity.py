@@ -43,6 +43,9 @@ def x_np(x):
     (128, "float16", tq.LAYOUT_ROW, 77),
     (192, "float16", tq.LAYOUT_BLOCK32, 555),
     (64, "float32", tq.LAYOUT_ROW, 300),
+    (100, "float32", tq.LAYOUT_BLOCK32, 333),  # d_pad 128, 400-byte rows (thread-per-vector)
+    (104, "float16", tq.LAYOUT_ROW, 129),      # d_pad 128 with 24 zero-filled columns (tensor core)
+    (36, "float32", tq.LAYOUT_ROW, 70),        # d_pad 64: warp-per-vector
 ])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_encode_mse_parity(d, dtype, layout, n, bits):
@@ -211,7 +214,10 @@ def _pack_cache(ora_k, ora_v, K, V, seq, cap):
 @pytest.mark.parametrize("d,G,seq,cap,bits,m", [(128, 8, 300, 320, 3, None), (128, 4, 64, 64, 2, None),
                                                 (192, 4, 1000, 1024, 4, None), (128, 1, 33, 64, 3, None),
                                                 (128, 4, 1000, 1024, 3, 64), (128, 8, 97, 128, 2, 64),
-                                                (128, 2, 413, 416, 4, 64)])
+                                                (128, 2, 413, 416, 4, 64),
+                                                (128, 16, 100, 128, 3, None),  # G = 16: SIMT kernel
+                                                (128, 4, 1, 32, 2, None),      # a single token
+                                                (100, 4, 77, 96, 3, None)])    # d = 100 padded to 128
 def test_attention_on_oracle_cache(d, G, seq, cap, bits, m):
     # m = 64: the QJL projection with d / 2 rows (a storage variant with
     # 8 bytes of signs per token instead of 16)

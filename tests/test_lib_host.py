@@ -120,6 +120,8 @@ def test_encode_and_attention_validation_before_launch():
     assert lib.tq_encode_mse(h, fake, 0, 10, 128, 0, 0, 5, fake, fake, None, 0, None) == 1
     assert lib.tq_encode_mse(h, mis, 0, 10, 128, 0, 0, 0, fake, fake, None, 0, None) == 1
     assert lib.tq_encode_mse(h, fake, 0, 10, 100, 0, 0, 0, fake, fake, None, 0, None) == 1  # ld < d
+    h100 = _mse_handle(100)
+    assert lib.tq_encode_mse(h100.handle, fake, 1, 10, 100, 0, 0, 0, fake, fake, None, 0, None) == 1  # 200-B rows
     assert lib.tq_encode_mse(h, fake, 0, 10, 128, 3, 0, 0, fake, fake, None, 0, None) == 1  # 10 % 3
     assert lib.tq_encode_mse(h, fake, 0, 10, 128, 10, 5, 0, fake, fake, None, 0, None) == 1  # cap < len
     assert lib.tq_encode_mse(h, fake, 0, 10, 128, 10, 40, 1, fake, fake, None, 0, None) == 1  # cap % 32

@@ -123,12 +123,15 @@ struct SignMasks {
 
 // Load 8 consecutive coordinates [8c, 8c + 8) of the staged row (c < row_bytes/16 for
 // 16-bit types; fp32 uses two chunks) with D applied, as floats.
+// `chunks` = 16-byte chunks in the row; an fp32 row whose length is 4 mod 8
+// ends with half of an 8-coordinate group, whose upper half reads as zeros.
 template <typename T>
-__device__ __forceinline__ void load8(const unsigned char* row, int c, const SignMasks& sg, float (&o)[8]);
+__device__ __forceinline__ void load8(const unsigned char* row, int c, const SignMasks& sg, float (&o)[8],
+                                      int chunks);
 
 template <>
 __device__ __forceinline__ void load8<__half>(const unsigned char* row, int c, const SignMasks& sg,
-                                              float (&o)[8]) {
+                                              float (&o)[8], int) {
   uint4 w = *reinterpret_cast<const uint4*>(row + c * 16);
   w.x ^= sg.m[4 * c + 0];
   w.y ^= sg.m[4 * c + 1];
@@ -145,7 +148,7 @@ __device__ __forceinline__ void load8<__half>(const unsigned char* row, int c, c
 
 template <>
 __device__ __forceinline__ void load8<__nv_bfloat16>(const unsigned char* row, int c,
-                                                     const SignMasks& sg, float (&o)[8]) {
+                                                     const SignMasks& sg, float (&o)[8], int) {
   uint4 w = *reinterpret_cast<const uint4*>(row + c * 16);
   w.x ^= sg.m[4 * c + 0];
   w.y ^= sg.m[4 * c + 1];
@@ -161,12 +164,13 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const unsigned char* row, i
 
 template <>
 __device__ __forceinline__ void load8<float>(const unsigned char* row, int c, const SignMasks& sg,
-                                             float (&o)[8]) {
+                                             float (&o)[8], int chunks) {
   const uint4 a = *reinterpret_cast<const uint4*>(row + c * 32);
-  const uint4 b = *reinterpret_cast<const uint4*>(row + c * 32 + 16);
+  const bool full = 2 * c + 1 < chunks;
+  const uint4 b = full ? *reinterpret_cast<const uint4*>(row + c * 32 + 16) : make_uint4(0u, 0u, 0u, 0u);
   const uint32_t ws[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) o[i] = __uint_as_float(ws[i] ^ sg.m[8 * c + i]);
+  for (int i = 0; i < 8; ++i) o[i] = __uint_as_float(ws[i] ^ (i < 4 || full ? sg.m[8 * c + i] : 0u));
 }
 
 // ------------------------------------------------------------------ quantize + pack
@@ -469,12 +473,12 @@ __global__ void __launch_bounds__(kThreads, 1) encode_kernel(QParams qp, SignMas
         float lo8[8], hi8[8];
         const bool in_lo = ESZ == 2 ? (c < chunks) : (2 * c < chunks);
         const bool in_hi = HALVES == 2 && (ESZ == 2 ? (c + 16 < chunks) : (2 * (c + 16) < chunks));
-        if (in_lo) load8<T>(row, c, sg, lo8);
+        if (in_lo) load8<T>(row, c, sg, lo8, chunks);
         else {
 #pragma unroll
           for (int i = 0; i < 8; ++i) lo8[i] = 0.f;
         }
-        if (in_hi) load8<T>(row, c + 16, sg, hi8);
+        if (in_hi) load8<T>(row, c + 16, sg, hi8, chunks);
         else {
 #pragma unroll
           for (int i = 0; i < 8; ++i) hi8[i] = 0.f;
