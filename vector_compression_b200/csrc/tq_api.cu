@@ -338,8 +338,10 @@ size_t attention_workspace(const QParams& kp, const QParams& vp, int L, int B, i
                            int64_t seq, int* chunk_out, int* n_chunks_out) {
   const int64_t groups = (int64_t)L * B * Hkv;
   const int G = Hq / Hkv;
-  const int64_t target = (int64_t)num_sms() * 32;
-  int64_t n_chunks = std::max<int64_t>(1, ceil_div(target, std::max<int64_t>(groups, 1)));
+  // about 28 CTAs per SM in all (seven waves of the int8 kernel's four CTAs
+  // per SM), rounding the chunk count down so the last wave stays full
+  const int64_t target = (int64_t)num_sms() * 28;
+  int64_t n_chunks = std::max<int64_t>(1, target / std::max<int64_t>(groups, 1));
   int64_t chunk = round_up(ceil_div(seq, n_chunks), 64);
   chunk = std::max<int64_t>(chunk, 256);
   n_chunks = ceil_div(seq, chunk);

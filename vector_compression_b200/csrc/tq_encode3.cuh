@@ -309,19 +309,33 @@ __device__ __forceinline__ void quant32_mse(const uint32_t (&ur)[32], const floa
       const float a = fabsf(u);
       S = shift_in(S, sub_bits(0.0f, u));
       if (DOT) sa += a;
+      // DOT: the differences in plain C, so that |u| and |d| fold into the
+      // additions as operand modifiers (same rounding as sub_bits)
       if (K >= 2) {
-        const uint32_t d0 = sub_bits(t[0], a);
+        uint32_t d0;
+        if (DOT) {
+          const float f = t[0] - a;
+          d0 = __float_as_uint(f);
+          D0 += fabsf(f);
+        } else {
+          d0 = sub_bits(t[0], a);
+        }
         T0 = shift_in(T0, d0);
-        if (DOT) D0 += fabsf(__uint_as_float(d0));
       }
       if (K >= 3) {
-        const uint32_t d1 = sub_bits(t[1], a), d2 = sub_bits(t[2], a);
+        uint32_t d1, d2;
+        if (DOT) {
+          const float f1 = t[1] - a, f2 = t[2] - a;
+          d1 = __float_as_uint(f1);
+          d2 = __float_as_uint(f2);
+          D1 += fabsf(f1);
+          D2 += fabsf(f2);
+        } else {
+          d1 = sub_bits(t[1], a);
+          d2 = sub_bits(t[2], a);
+        }
         T1 = shift_in(T1, d1);
         T2 = shift_in(T2, d2);
-        if (DOT) {
-          D1 += fabsf(__uint_as_float(d1));
-          D2 += fabsf(__uint_as_float(d2));
-        }
       }
     }
     M0 = K == 3 ? (T0 ^ T1 ^ T2) : T0;
