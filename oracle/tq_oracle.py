@@ -24,8 +24,7 @@ Sources (page titles as given; sections / equations on each page):
 * [FVQ]    FastVQ README (Zapdev-labs/turboquant): sign-flipped Hadamard
   backend and padding of the trailing dimension.
 
-Readings taken where the pages are silent or garbled (each listed in
-DESIGN.md):
+Readings taken where the pages are silent or garbled:
 
 * Codebook for a padded Hadamard vector uses d = d_pad.
 * Rotation: y = H (D * pad(x)) / sqrt(d_pad), H the Sylvester matrix in
