@@ -50,6 +50,10 @@ def parse():
     ap.add_argument("--value-scale", default="norm", choices=["norm", "unbiased"],
                     help="per-vector scale stored with the values: the norm, or EDEN's unbiased scale")
     ap.add_argument("--rnorm-f16", action="store_true", help="store the keys' residual norms as fp16")
+    ap.add_argument("--retrieval-queries", type=int, default=0,
+                    help="instead of the KV-cache step, time the retrieval set (1e6 x 1536 unit vectors, dense "
+                         "rotation): Q_prod encode of the whole set and scores + top-10 for this many queries")
+    ap.add_argument("--retrieval-bits", type=int, default=2, choices=[2, 4])
     ap.add_argument("--qjl-rows", type=int, default=0,
                     help="QJL projection rows m of the keys (0 = the padded head dim; d_pad / 2 is the half-size variant)")
     return ap.parse_args()
@@ -231,8 +235,68 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+def run_retrieval(args):
+    """Retrieval set timing (one GPU): Q_prod encode of 1e6 x 1536 fp32 unit
+    vectors with the dense rotation (y = Pi x and z = S r are dense
+    contractions, 2 d^2 + 2 m d flop per vector), then scores for the first
+    `--retrieval-queries` queries and their top-10 (2 (d + m) flop per pair).
+    Prints one JSON line with both parts."""
+    import torch
+
+    import vector_compression_b200 as tq
+
+    R = synth.RETRIEVAL
+    n, d, m, bits = R["n"], R["d"], R["m"], args.retrieval_bits
+    dr = synth.method_draws(d, m, R["seed"], dense=True)
+    p = tq.TQParams(d, bits, tq.MODE_PROD, tq.ROT_DENSE, m=m, S=dr["S"], G=dr["G"])
+    dev = torch.device("cuda", 0)
+    x = synth.gaussian_vectors(n, d, seed=R["seed"], device=dev, n_outliers=R["n_outliers"],
+                               outlier_scale=R["outlier_scale"], normalize=True)
+    nq = args.retrieval_queries
+    q = synth.gaussian_vectors(nq, d, seed=R["seed"] + 1, device=dev, normalize=True)
+    out = (torch.empty((n, p.code_words), dtype=torch.int32, device=dev),
+           torch.empty((n, p.sign_words), dtype=torch.int32, device=dev),
+           torch.empty(n, dtype=torch.float32, device=dev), torch.empty(n, dtype=torch.float32, device=dev))
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    enc_ms = timed(lambda: tq.tq_encode_prod(p, x, out=out), args.steps)
+    sc_ms = timed(lambda: tq.tq_scores(p, q, *out, topk=R["topk"]), max(1, args.steps // 5))
+    tq.tq_sync_check()
+    enc_bytes = n * (d * 4 + 4 * (p.code_words + p.sign_words) + 8)
+    enc_flop = n * (2 * d * d + 2 * m * d)
+    sc_flop = nq * n * 2 * (d + m)
+    peak_tf = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] \
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1590.0
+    line = {
+        "metric": "retrieval set: Q_prod encode and scores + top-10", "workload": "retrieval 1e6 x 1536, dense",
+        "bits": bits, "m": m, "queries": nq,
+        "encode": {"ms": enc_ms, "GB/s": enc_bytes / (enc_ms * 1e-3) / 1e9,
+                   "TFLOP/s": enc_flop / (enc_ms * 1e-3) / 1e12,
+                   "frac_of_bf16_peak": enc_flop / (enc_ms * 1e-3) / 1e12 / peak_tf},
+        "scores_topk": {"ms": sc_ms, "TFLOP/s": sc_flop / (sc_ms * 1e-3) / 1e12,
+                        "frac_of_bf16_peak": sc_flop / (sc_ms * 1e-3) / 1e12 / peak_tf,
+                        "pairs_per_s": nq * n / (sc_ms * 1e-3)},
+        "arithmetic": "fp32 (CUDA cores); the peak is the measured bf16 tensor figure",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    if args.retrieval_queries:
+        return run_retrieval(args)
     cfg = synth.KV_CONFIGS[args.workload]
     if args.layers:
         cfg = cfg.scaled(layers=min(args.layers, cfg.layers))

@@ -343,6 +343,12 @@ size_t attention_workspace(const QParams& kp, const QParams& vp, int L, int B, i
   const int64_t target = (int64_t)num_sms() * 28;
   int64_t n_chunks = std::max<int64_t>(1, target / std::max<int64_t>(groups, 1));
   int64_t chunk = round_up(ceil_div(seq, n_chunks), 64);
+  if (chunk < 1024) {
+    // short chunks would spend most of a CTA on its per-query setup: aim at
+    // one wave of CTAs instead
+    n_chunks = std::max<int64_t>(1, (int64_t)num_sms() * 4 / std::max<int64_t>(groups, 1));
+    chunk = round_up(ceil_div(seq, n_chunks), 64);
+  }
   chunk = std::max<int64_t>(chunk, 256);
   n_chunks = ceil_div(seq, chunk);
   if (chunk_out) *chunk_out = (int)chunk;
