@@ -30,7 +30,7 @@ PFN_cuTensorMapEncodeTiled encode_tiled_fn() {
 int prod_tpr() {
   static const int tpr = [] {
     const char* e = getenv("TQ_PROD_TPR");
-    return (e && e[0] == '4') ? 4 : 2;
+    return (e && e[0] == '4') ? 4 : (e && e[0] == '2') ? 2 : 1;
   }();
   return tpr;
 }

@@ -1008,5 +1008,294 @@ __global__ void __launch_bounds__(prod_threads<TPR>(), 1)
   }
 }
 
+// ------------------------------------------------------------------ Q_prod, one thread per vector
+
+// Q_prod with the Q_MSE kernel's work split: two epilogue groups of four
+// warps take alternate tiles (group g the tiles L = g mod 2, in TMEM buffer
+// g), and thread (warp w, lane l) owns TMEM lane 32 (w % 4) + l, i.e. one
+// whole vector: its norm, quantization, residual and signs need no exchange
+// between threads.  Per tile a group: reads u (two 32-column chunks at a
+// time for the norm, then chunk by chunk), writes 2^10 r as fp16 hi + lo over
+// u, signals the MMA warp, stores
+// codes and norms, then waits for z = S r and packs the signs; while it waits
+// for the MMA, the other group's warps on the same sub-partitions quantize
+// the next tile.  The MMA warp issues u = (H D) x of tile L, then S r of
+// tile L - 1.  Every wait is bounded (error word + clean exit).
+template <typename T, int K>
+__global__ void __launch_bounds__(kThreads, 1)
+    encode_prod_rows_kernel(const __grid_constant__ CUtensorMap xmap, QParams qp, Args a) {
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages];
+  __shared__ __align__(8) uint64_t bar_accf[2], bar_aready[2], bar_zf[2], bar_done;
+  __shared__ uint32_t tmem_base_s;
+  constexpr bool BF16 = !std::is_same<T, __half>::value;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m = qp.m;
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  unsigned char* rot = smem;
+  unsigned char* smat = smem + kRotBytes;
+  unsigned char* stages = smat + m * kDP * 2;
+  constexpr uint32_t tmem_cols = 512u;
+
+  // ---- setup: rotation operand H D (+-1), S (fp16), barriers, TMEM
+  {
+    const uint16_t one = BF16 ? 0x3F80u : 0x3C00u;
+    for (int e = tid; e < kDP * (kDP / 8); e += kThreads) {
+      const int n = e / (kDP / 8), kc = e % (kDP / 8);
+      uint16_t v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int k = kc * 8 + i;
+        const uint32_t neg = (__popc(n & k) & 1) ^ ((qp.dmask[k >> 5] >> (k & 31)) & 1u);
+        v[i] = (uint16_t)(one | (neg << 15));
+      }
+      uint4 w;
+      w.x = v[0] | ((uint32_t)v[1] << 16);
+      w.y = v[2] | ((uint32_t)v[3] << 16);
+      w.z = v[4] | ((uint32_t)v[5] << 16);
+      w.w = v[6] | ((uint32_t)v[7] << 16);
+      *reinterpret_cast<uint4*>(rot + core_offset(n, kc * 8, kDP)) = w;
+    }
+    for (int e = tid; e < m * (kDP / 8); e += kThreads) {
+      const int row = e / (kDP / 8), kc = e % (kDP / 8);
+      const uint4 w = *reinterpret_cast<const uint4*>(qp.S16 + (size_t)row * kDP + kc * 8);
+      *reinterpret_cast<uint4*>(smat + core_offset(row, kc * 8, m)) = w;
+    }
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&bar_full[s]), 1);
+      mbar_init(smem_u32(&bar_empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bar_accf[b]), 1);
+      mbar_init(smem_u32(&bar_aready[b]), 128);  // every thread of the group
+      mbar_init(smem_u32(&bar_zf[b]), 1);
+    }
+    mbar_init(smem_u32(&bar_done), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_base_s)),
+                 "r"(tmem_cols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  const int64_t G = gridDim.x;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int L = 0;; ++L) {
+        const int64_t tile = blockIdx.x + (int64_t)L * G;
+        if (tile >= a.n_tiles) break;
+        const int s = L % kStages;
+        if (L >= kStages && !mbar_wait(smem_u32(&bar_empty[s]), ((L / kStages) - 1) & 1, a.err)) break;
+        const uint32_t dst = smem_u32(stages + s * kTileBytes);
+        mbar_arrive_tx(smem_u32(&bar_full[s]), kTileBytes);
+        tma_load_2d(dst, &xmap, 0, (int)(tile * kRows), smem_u32(&bar_full[s]));
+        tma_load_2d(dst + kTileBytes / 2, &xmap, 64, (int)(tile * kRows), smem_u32(&bar_full[s]));
+        issued = L + 1;
+      }
+      for (int L = issued - kStages < 0 ? 0 : issued - kStages; L < issued; ++L)
+        mbar_wait(smem_u32(&bar_full[L % kStages]), (L / kStages) & 1, a.err);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t fmt = BF16 ? 1u : 0u;
+      const uint32_t idesc1 = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kDP >> 3) << 17) |
+                              ((uint32_t)(kRows >> 4) << 24);
+      const uint32_t idesc2 = (1u << 4) | ((uint32_t)(m >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
+      const uint32_t rot_base = smem_u32(rot);
+      const uint32_t s_base = smem_u32(smat);
+      const uint32_t s_lbo = (uint32_t)(m / 8) * 128u;
+      for (int L = 0;; ++L) {
+        const int64_t tile = blockIdx.x + (int64_t)L * G;
+        const bool have = tile < a.n_tiles;
+        if (have) {
+          // u of tile L into buffer L & 1; the residual of tile L - 2 that it
+          // overwrites was read by the S r MMA issued before this one
+          const int s = L % kStages, b = L & 1;
+          if (!mbar_wait(smem_u32(&bar_full[s]), (L / kStages) & 1, a.err)) break;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(stages + s * kTileBytes);
+          const uint32_t d_tmem = tmem + (uint32_t)b * 256u;
+#pragma unroll
+          for (int t = 0; t < kDP / 16; ++t) {
+            const uint64_t ad = desc_sw128(a_base + (uint32_t)(t >> 2) * (kTileBytes / 2) + (uint32_t)(t & 3) * 32u);
+            const uint64_t bd = desc_noswz(rot_base + (uint32_t)(2 * t) * 2048u, 2048u, 128u);
+            mma_ss(d_tmem, ad, bd, idesc1, t > 0 ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&bar_empty[s]));
+          tc_commit(smem_u32(&bar_accf[b]));
+        }
+        if (L >= 1) {
+          // z = S r of tile L - 1 once its group has written the residual (the
+          // group read the previous z of this buffer before that)
+          const int Lp = L - 1, b = Lp & 1;
+          if (!mbar_wait(smem_u32(&bar_aready[b]), (Lp >> 1) & 1, a.err)) break;
+          tc_fence_after();
+          const uint32_t a_tmem = tmem + (uint32_t)b * 256u;
+          const uint32_t z_tmem = a_tmem + 128u;
+#pragma unroll
+          for (int pass = 0; pass < 2; ++pass) {  // hi, then lo parts of r
+#pragma unroll
+            for (int t = 0; t < kDP / 16; ++t) {
+              const uint32_t acol = (uint32_t)(32 * (t >> 1) + 16 * pass + 8 * (t & 1));
+              const uint64_t bd = desc_noswz(s_base + (uint32_t)(2 * t) * s_lbo, s_lbo, 128u);
+              mma_ts(z_tmem, a_tmem + acol, bd, idesc2, (pass | t) ? 1u : 0u);
+            }
+          }
+          tc_commit(smem_u32(&bar_zf[b]));
+        }
+        if (!have) break;
+      }
+      tc_commit(smem_u32(&bar_done));
+      mbar_wait(smem_u32(&bar_done), 0, a.err);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue groups
+    const int grp = (warp - 2) >> 2;  // 0 or 1: tiles L = grp mod 2, TMEM buffer grp
+    const int quarter = warp & 3;     // TMEM lanes 32*quarter .. +31
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t ubase = tmem + (uint32_t)grp * 256u + lane_off;
+    const int half_levels = 1 << (K - 1);
+    float tc[4], dc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tc[j] = dc[j] = 0.f;
+    const float c0s = 1024.0f * qp.centroids[half_levels];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      if (j < half_levels - 1) {
+        tc[j] = 1024.0f * qp.boundaries[half_levels + j] - c0s;
+        dc[j] = 1024.0f * (qp.centroids[half_levels + j + 1] - qp.centroids[half_levels + j]);
+      }
+    }
+    const int sw_words = m / 32;  // sign words per vector (2 or 4)
+    for (int L = grp;; L += 2) {
+      const int64_t tile = blockIdx.x + (int64_t)L * G;
+      if (tile >= a.n_tiles) break;
+      const uint32_t par = (uint32_t)(L >> 1) & 1u;
+      if (!mbar_wait_warp(smem_u32(&bar_accf[grp]), par, a.err)) break;
+      tc_fence_after();
+      const int64_t row = tile * kRows + quarter * 32 + lane;
+      const bool valid = row < a.n_vec;
+      const int64_t seg = valid ? (int64_t)fastdiv((uint32_t)row, a.seg_div) : 0;
+      const int64_t slot = seg * a.seg_cap + (valid ? row - seg * a.seg_len : 0);
+
+      // pass 1: ||u|| over the four chunks
+      uint32_t ra[32], rb[32];
+      uint64_t s2a = 0, s2b = 0;
+      auto sumsq = [&](const uint32_t (&r)[32]) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const uint64_t p0 = pk2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+          const uint64_t p1 = pk2(__uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
+          s2a = fma2(p0, p0, s2a);
+          s2b = fma2(p1, p1, s2b);
+        }
+      };
+      tmem_ld32(ubase, ra);
+      tmem_ld32(ubase + 32u, rb);
+      tmem_ld_wait2(ra, rb);
+      sumsq(ra);
+      sumsq(rb);
+      tmem_ld32(ubase + 64u, ra);
+      tmem_ld32(ubase + 96u, rb);
+      tmem_ld_wait2(ra, rb);
+      sumsq(ra);
+      sumsq(rb);
+      const float2 fa = upk2(s2a), fb = upk2(s2b);
+      const float ss = (fa.x + fa.y) + (fb.x + fb.y);  // ||u||^2 = d_pad ||x||^2
+      const bool zero = !(ss > 0.f);
+      const float rs = rsqrtf(ss);
+      const float nu = zero ? 0.f : ss * rs;
+      const float inv = zero ? 0.f : 1024.0f * rs;
+
+      // pass 2: quantize chunk c, write 2^10 r as fp16 hi (columns 32c .. 32c+15)
+      // and lo (32c+16 .. 32c+31) over u
+      uint64_t rr2 = 0;
+      uint32_t* dst = a.codes + slot * (int64_t)(K * 4);
+      auto process = [&](const int c, uint32_t (&r)[32]) {
+        float (&v)[32] = *reinterpret_cast<float(*)[32]>(&r);  // quantized in place
+        uint32_t NS = 0, T0 = 0, T1 = 0, T2 = 0;
+        quant32_prod_sb<K>(v, tc, dc, c0s, inv, NS, T0, T1, T2);
+        if (valid) {  // word c of every plane
+          const uint32_t S = zero ? 0u : ~NS;
+          const uint32_t M0 = K == 3 ? (T0 ^ T1 ^ T2) : T0;
+          uint32_t planes[K];
+          planes_from<K>(S, M0, T1, 0u, planes);
+#pragma unroll
+          for (int p = 0; p < K; ++p) dst[4 * p + c] = planes[p];
+        }
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          uint32_t hiw[8], low[8];
+#pragma unroll
+          for (int qq = 0; qq < 8; ++qq) {
+            const float r0 = v[16 * g + 2 * qq], r1 = v[16 * g + 2 * qq + 1];
+            const float h0 = __uint_as_float(__float_as_uint(r0) & 0xFFFFE000u);
+            const float h1 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
+            const uint64_t rp = pk2(r0, r1);
+            rr2 = fma2(rp, rp, rr2);
+            const float2 lo = upk2(sub2(rp, pk2(h0, h1)));
+            const __half2 hv = __floats2half2_rn(h0, h1);
+            const __half2 lv = __floats2half2_rn(lo.x, lo.y);
+            hiw[qq] = *reinterpret_cast<const uint32_t*>(&hv);
+            low[qq] = *reinterpret_cast<const uint32_t*>(&lv);
+          }
+          tmem_st8(ubase + (uint32_t)(32 * c + 8 * g), hiw);
+          tmem_st8(ubase + (uint32_t)(32 * c + 16 + 8 * g), low);
+        }
+      };
+      // every chunk reloaded (a chunk's columns are rewritten only after it
+      // has been loaded); the other group's warps cover the load latency
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32_sync(ubase + (uint32_t)(32 * c), ra);
+        process(c, ra);
+      }
+      const float2 rrf = upk2(rr2);
+      const float rr = rrf.x + rrf.y;
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(smem_u32(&bar_aready[grp]));
+      if (valid) {
+        a.norms[slot] = nu * qp.inv_sqrt_dpad;
+        put_rnorm(a.rnorms, slot, rr > 0.f ? rr * rsqrtf(rr) * (1.0f / 1024.0f) : 0.f, qp.rnorm_f16);
+      }
+      // signs of this tile once z = S r is in TMEM (the other group's warps
+      // keep the sub-partitions busy meanwhile)
+      if (!mbar_wait_warp(smem_u32(&bar_zf[grp]), par, a.err)) break;
+      tc_fence_after();
+      for (int c = 0; c < sw_words; ++c) {
+        uint32_t z[32];
+        tmem_ld32_sync(tmem + (uint32_t)grp * 256u + 128u + (uint32_t)(32 * c) + lane_off, z);
+        uint32_t neg = 0;
+#pragma unroll
+        for (int i = 31; i >= 0; --i) neg = shift_in(neg, z[i]);
+        // bit i = [(S r)_(32c+i) >= 0]; a zero vector's residual was formed
+        // with the opposite sign (see quant32_prod_sb)
+        if (valid) a.signs[slot * sw_words + c] = zero ? neg : ~neg;
+      }
+      tc_fence_before();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols));
+  }
+}
+
 }  // namespace enc3
 }  // namespace tq
