@@ -1257,7 +1257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // every chunk reloaded (a chunk's columns are rewritten only after it
       // has been loaded); the other group's warps cover the load latency
-#pragma unroll 1
+#pragma unroll 2
       for (int c = 0; c < 4; ++c) {
         tmem_ld32_sync(ubase + (uint32_t)(32 * c), ra);
         process(c, ra);
