@@ -360,9 +360,11 @@ size_t attention_workspace(const QParams& kp, const QParams& vp, int L, int B, i
 }
 
 // The tensor-core kernels (int8: tq_attn3.cu, fp16: tq_attn2.cu) cover
-// d_pad = 128, m = 128, at most 8 query heads per KV head and key codes of
-// 1..3 bits; the int8 kernel runs unless TQ_ATTN_V2=1 selects the fp16 one,
-// and TQ_ATTN_V1=1 selects the SIMT kernel for every shape.
+// at most 8 query heads per KV head and key codes of 1..3 bits: the int8
+// kernel d_pad = 128 with m = 64 or 128 and d_pad = 256 with m = 256, the
+// fp16 kernel d_pad = 128 with m = 128.  The int8 kernel runs unless
+// TQ_ATTN_V2=1 selects the fp16 one, and TQ_ATTN_V1=1 selects the SIMT kernel
+// for every shape.
 static const bool g_attn_v2 = [] {
   const char* e = getenv("TQ_ATTN_V1");
   return !(e && e[0] == '1');
@@ -372,10 +374,10 @@ static const bool g_attn_v3 = [] {
   return g_attn_v2 && !(e && e[0] == '1');
 }();
 
-// m = 128 for the fp16 kernel; the int8 kernel also takes m = 64
 static bool attn2_covers(const QParams& kp, const QParams& vp, int G) {
-  return g_attn_v2 && kp.rot == TQ_ROT_HADAMARD && kp.d_pad == 128 && vp.d_pad == 128 &&
-         (kp.m == 128 || (kp.m == 64 && g_attn_v3)) && G >= 1 && G <= 8 && kp.k >= 1 && kp.k <= 3 &&
+  const bool shape = (kp.d_pad == 128 && vp.d_pad == 128 && (kp.m == 128 || (kp.m == 64 && g_attn_v3))) ||
+                     (kp.d_pad == 256 && vp.d_pad == 256 && kp.m == 256 && g_attn_v3);
+  return g_attn_v2 && kp.rot == TQ_ROT_HADAMARD && shape && G >= 1 && G <= 8 && kp.k >= 1 && kp.k <= 3 &&
          vp.k >= 1 && vp.k <= 4;
 }
 
@@ -432,8 +434,8 @@ int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q
                     aligned16(vnorms);
     cudaError_t ce = cudaErrorInvalidValue;
     if (v3)
-      ce = attn3::launch(p2, kp.k, vp.k, kp.m, grid, st);
-    else if (kp.m == 128)
+      ce = attn3::launch(p2, kp.k, vp.k, kp.m, kp.d_pad, grid, st);
+    else if (kp.m == 128 && kp.d_pad == 128)
       ce = attn2::launch(p2, kp.k, vp.k, grid, st);
     if (ce != cudaSuccess) return ce;
   } else {

@@ -121,9 +121,13 @@ __device__ __forceinline__ uint32_t fixed_byte(float x, float inv, int piece) {
 // Shared-memory layout of one CTA (bytes): the staged sub-chunk (key codes,
 // sign words, key norms, residual norms | value blocks, value norms), scores
 // (which first hold the query rows during setup) and weight bytes.
-template <int KK, int KV, int NT, int MQ>
+template <int KK, int KV, int NT, int MQ, int DPT>
 struct Layout {
+  // d_pad 256: one warp per 32 value coordinates (eight warps) and 192-token
+  // sub-chunks; the query fragments live in shared memory
+  static constexpr int DP = DPT, WPP = DPT / 32, SC = DPT == 128 ? 384 : 192;
   static constexpr int KW = KK * WPP, HN = 4 * NT, SW = MQ / 32;
+  static constexpr int SROWS = SC > 2 * DP ? SC : 2 * DP;  // score rows (query rows during setup)
   static constexpr uint32_t kc = 0;
   static constexpr uint32_t ks = kc + SC * KW * 4;
   static constexpr uint32_t kn = ks + SC * SW * 4;
@@ -131,11 +135,12 @@ struct Layout {
   static constexpr uint32_t vc = kr + SC * 4;
   static constexpr uint32_t vn = vc + (SC / 32) * KV * DP * 4;
   static constexpr uint32_t score = vn + SC * 4;
-  static constexpr uint32_t wb = score + SC * HN * 4;
-  static constexpr uint32_t bytes = wb + (SC / 32) * NT * 8 * 4 * 2 * 4;
+  static constexpr uint32_t wb = score + SROWS * HN * 4;
+  static constexpr uint32_t bq = wb + (SC / 32) * NT * 8 * 4 * 2 * 4;
+  static constexpr uint32_t bytes = bq + (DPT == 128 ? 0 : (NT + 1) * 2 * WPP * 32 * 8);
   // the query rows (setup only) share the score buffer
   static constexpr uint32_t qf = score;
-  static_assert(SC * HN >= 2 * HN * DP, "query rows fit in the score buffer");
+  static_assert(SROWS * HN >= 2 * HN * DP, "query rows fit in the score buffer");
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -171,10 +176,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   }
 }
 
-template <int KK, int KV, int NT, int MQ>
-__global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
-  using LY = Layout<KK, KV, NT, MQ>;
-  constexpr int SW = MQ / 32;    // QJL sign words per token (m = 64 or 128)
+template <int KK, int KV, int NT, int MQ, int DPT>
+__global__ void __launch_bounds__(DPT) attn_kernel(Params P) {
+  using LY = Layout<KK, KV, NT, MQ, DPT>;
+  // geometry of this d_pad (shadows the d_pad = 128 constants above)
+  constexpr int DP = LY::DP, WPP = LY::WPP, SC = LY::SC;
+  constexpr int kWarps = DPT / 32, kThreads = DPT;
+  constexpr int SW = MQ / 32;    // QJL sign words per token (m / 32)
   constexpr int FK = NF<KK>::v;  // key code features
   constexpr int FV = NF<KV>::v;  // value code features
   constexpr int KW = KK * WPP;   // key code words per token
@@ -192,6 +200,7 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
   static_assert(LY::score % 16 == 0, "vector access to the score rows");
   uint32_t (*s_wb)[NT][8][4][2] = reinterpret_cast<uint32_t (*)[NT][8][4][2]>(smem + LY::wb);
   float (*s_qf)[HN][DP] = reinterpret_cast<float (*)[HN][DP]>(smem + LY::qf);
+  uint2 (*s_bq)[2][WPP][32] = reinterpret_cast<uint2 (*)[2][WPP][32]>(smem + LY::bq);  // d_pad 256
   __shared__ __align__(8) uint64_t bar_k, bar_v;
   __shared__ float s_red[3][kWarps][HN];
   __shared__ float s_head[HN][8];  // per head: Qq, Qu, sum q_int, sum u_int, m, l, 1/Qq, 1/Qu
@@ -251,12 +260,12 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
     const int which = hw / HN, h = hw % HN;
     float mx = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) mx = fmaxf(mx, fabsf(s_qf[which][h][lane + 32 * i]));
+    for (int i = 0; i < WPP; ++i) mx = fmaxf(mx, fabsf(s_qf[which][h][lane + 32 * i]));
     mx = warp_max(mx);
     const float inv = mx > 0.f ? kQMax / mx : 0.f;
-    int sum = 0;  // |sum| <= 128 * 127 * 2^16 < 2^31
+    int sum = 0;  // |sum| <= d_pad * 127 * 2^16 < 2^31 for d_pad <= 256
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sum += __float2int_rn(s_qf[which][h][lane + 32 * i] * inv);
+    for (int i = 0; i < WPP; ++i) sum += __float2int_rn(s_qf[which][h][lane + 32 * i] * inv);
     sum = __reduce_add_sync(0xffffffffu, sum);
     if (lane == 0) {
       s_head[h][which] = mx / kQMax;      // Qq or Qu
@@ -273,29 +282,44 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
   // even) or mid; of tile NT: head g / 2 (g even) or 4 + g / 2, piece lo.  For
   // plane word cw, b0 bytes = coordinates 32 cw + 2 tig + 8 i and b1 =
   // 32 cw + 2 tig + 1 + 8 i.
-  uint32_t bq[NT + 1][2][WPP][2];
+  // d_pad 128: in registers; d_pad 256: in shared memory (the same for every
+  // warp; warp 0 writes them)
+  uint32_t bq[DPT == 128 ? NT + 1 : 1][2][DPT == 128 ? WPP : 1][2];
+  if (DPT == 128 || warp == 0) {
 #pragma unroll
-  for (int nt = 0; nt <= NT; ++nt) {
-    const int hc = nt < NT ? 4 * nt + (g >> 1) : (g & 1) * 4 + (g >> 1);
-    const bool hv = hc < HN;  // lo tile with one head tile: columns of heads 4..7 are zero
-    const int h = hv ? hc : 0;
-    const int piece = nt < NT ? (g & 1) : 2;
+    for (int nt = 0; nt <= NT; ++nt) {
+      const int hc = nt < NT ? 4 * nt + (g >> 1) : (g & 1) * 4 + (g >> 1);
+      const bool hv = hc < HN;  // lo tile with one head tile: columns of heads 4..7 are zero
+      const int h = hv ? hc : 0;
+      const int piece = nt < NT ? (g & 1) : 2;
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const float inv = s_head[h][6 + which];
+      for (int which = 0; which < 2; ++which) {
+        const float inv = s_head[h][6 + which];
 #pragma unroll
-      for (int cw = 0; cw < WPP; ++cw) {
+        for (int cw = 0; cw < WPP; ++cw) {
+          uint32_t w2[2];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          uint32_t w = 0;
+          for (int r = 0; r < 2; ++r) {
+            uint32_t w = 0;
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            w |= fixed_byte(s_qf[which][h][32 * cw + 2 * tig + r + 8 * i], inv, piece) << (8 * i);
-          bq[nt][which][cw][r] = hv ? w : 0u;
+            for (int i = 0; i < 4; ++i)
+              w |= fixed_byte(s_qf[which][h][32 * cw + 2 * tig + r + 8 * i], inv, piece) << (8 * i);
+            w2[r] = hv ? w : 0u;
+          }
+          if constexpr (DPT == 128) {
+            bq[nt][which][cw][0] = w2[0];
+            bq[nt][which][cw][1] = w2[1];
+          } else {
+            s_bq[nt][which][cw][lane] = make_uint2(w2[0], w2[1]);
+          }
         }
       }
     }
   }
+  auto bfrag = [&](int nt, int which, int cw) -> uint2 {
+    if constexpr (DPT == 128) return make_uint2(bq[nt][which][cw][0], bq[nt][which][cw][1]);
+    else return s_bq[nt][which][cw][lane];
+  };
   __syncthreads();  // the query rows (in the score buffer) have been read
   // per thread-column heads (4 nt + tig): score constants, log2 domain
   float cA1[NT], cC1[NT], cA2[NT], cC2[NT];
@@ -337,11 +361,14 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
         k1[i] = a.x; k1[i + 1] = a.y; k1[i + 2] = a.z; k1[i + 3] = a.w;
         k2[i] = b.x; k2[i + 1] = b.y; k2[i + 2] = b.z; k2[i + 3] = b.w;
       }
-      if (SW == 4) {
-        const uint4 a = *reinterpret_cast<const uint4*>(s_ks + R1 * SW);
-        const uint4 b = *reinterpret_cast<const uint4*>(s_ks + R2 * SW);
-        k1[KW] = a.x; k1[KW + 1] = a.y; k1[KW + 2] = a.z; k1[KW + 3] = a.w;
-        k2[KW] = b.x; k2[KW + 1] = b.y; k2[KW + 2] = b.z; k2[KW + 3] = b.w;
+      if (SW % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < SW; i += 4) {
+          const uint4 a = *reinterpret_cast<const uint4*>(s_ks + R1 * SW + i);
+          const uint4 b = *reinterpret_cast<const uint4*>(s_ks + R2 * SW + i);
+          k1[KW + i] = a.x; k1[KW + i + 1] = a.y; k1[KW + i + 2] = a.z; k1[KW + i + 3] = a.w;
+          k2[KW + i] = b.x; k2[KW + i + 1] = b.y; k2[KW + i + 2] = b.z; k2[KW + i + 3] = b.w;
+        }
       } else {
         const uint2 a = *reinterpret_cast<const uint2*>(s_ks + R1 * SW);
         const uint2 b = *reinterpret_cast<const uint2*>(s_ks + R2 * SW);
@@ -374,8 +401,10 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
           const uint32_t a2 = bits_to_bytes(W1, mul1), a3 = bits_to_bytes(W2, mul1);
           const int which = f < FK ? 0 : 1;
 #pragma unroll
-          for (int nt = 0; nt <= NT; ++nt)
-            mma_u8s8(acc[f][nt], a0, a1, a2, a3, bq[nt][which][cw][0], bq[nt][which][cw][1]);
+          for (int nt = 0; nt <= NT; ++nt) {
+            const uint2 bb = bfrag(nt, which, cw);
+            mma_u8s8(acc[f][nt], a0, a1, a2, a3, bb.x, bb.y);
+          }
         }
       }
       // s log2(e) = scale log2(e) n (Qq (sum_S alpha_S v_S / 64 - sum alpha sum q_int)
@@ -613,39 +642,44 @@ __global__ void __launch_bounds__(kThreads) attn_kernel(Params P) {
   }
 }
 
-template <int KK, int KV, int NT, int MQ>
+template <int KK, int KV, int NT, int MQ, int DPT>
 cudaError_t launch_nt(const Params& p, dim3 grid, cudaStream_t st) {
-  auto kern = attn_kernel<KK, KV, NT, MQ>;
-  const int smem = (int)Layout<KK, KV, NT, MQ>::bytes;
+  auto kern = attn_kernel<KK, KV, NT, MQ, DPT>;
+  const int smem = (int)Layout<KK, KV, NT, MQ, DPT>::bytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, st>>>(p);
+  kern<<<grid, DPT, smem, st>>>(p);
   return cudaGetLastError();
 }
 
+// d_pad 128 with m = 64 or 128; d_pad 256 with m = 256
 template <int KK, int KV>
-cudaError_t launch_kv(const Params& p, int m, dim3 grid, cudaStream_t st) {
-  if (m == 64) return p.G <= 4 ? launch_nt<KK, KV, 1, 64>(p, grid, st) : launch_nt<KK, KV, 2, 64>(p, grid, st);
-  return p.G <= 4 ? launch_nt<KK, KV, 1, 128>(p, grid, st) : launch_nt<KK, KV, 2, 128>(p, grid, st);
+cudaError_t launch_kv(const Params& p, int m, int dp, dim3 grid, cudaStream_t st) {
+  if (dp == 256)
+    return p.G <= 4 ? launch_nt<KK, KV, 1, 256, 256>(p, grid, st) : launch_nt<KK, KV, 2, 256, 256>(p, grid, st);
+  if (m == 64)
+    return p.G <= 4 ? launch_nt<KK, KV, 1, 64, 128>(p, grid, st) : launch_nt<KK, KV, 2, 64, 128>(p, grid, st);
+  return p.G <= 4 ? launch_nt<KK, KV, 1, 128, 128>(p, grid, st) : launch_nt<KK, KV, 2, 128, 128>(p, grid, st);
 }
 
 template <int KK>
-cudaError_t launch_k(const Params& p, int kv, int m, dim3 grid, cudaStream_t st) {
+cudaError_t launch_k(const Params& p, int kv, int m, int dp, dim3 grid, cudaStream_t st) {
   switch (kv) {
-    case 1: return launch_kv<KK, 1>(p, m, grid, st);
-    case 2: return launch_kv<KK, 2>(p, m, grid, st);
-    case 3: return launch_kv<KK, 3>(p, m, grid, st);
-    case 4: return launch_kv<KK, 4>(p, m, grid, st);
+    case 1: return launch_kv<KK, 1>(p, m, dp, grid, st);
+    case 2: return launch_kv<KK, 2>(p, m, dp, grid, st);
+    case 3: return launch_kv<KK, 3>(p, m, dp, grid, st);
+    case 4: return launch_kv<KK, 4>(p, m, dp, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch(const Params& p, int kk, int kv, int m, dim3 grid, cudaStream_t st) {
-  if (p.G < 1 || p.G > 8 || (m != 64 && m != 128)) return cudaErrorInvalidValue;
+cudaError_t launch(const Params& p, int kk, int kv, int m, int dp, dim3 grid, cudaStream_t st) {
+  if (p.G < 1 || p.G > 8) return cudaErrorInvalidValue;
+  if (!(dp == 128 && (m == 64 || m == 128)) && !(dp == 256 && m == 256)) return cudaErrorInvalidValue;
   switch (kk) {
-    case 1: return launch_k<1>(p, kv, m, grid, st);
-    case 2: return launch_k<2>(p, kv, m, grid, st);
-    case 3: return launch_k<3>(p, kv, m, grid, st);
+    case 1: return launch_k<1>(p, kv, m, dp, grid, st);
+    case 2: return launch_k<2>(p, kv, m, dp, grid, st);
+    case 3: return launch_k<3>(p, kv, m, dp, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
