@@ -348,6 +348,16 @@ tq_status tq_decode_step_workspace_size(const tq_params* kp, const tq_params* vp
  */
 tq_status tq_sync_check(void* stream);
 
+/*
+ * tq_check_wait_expiry -- exercise the bounded-wait path that every kernel
+ * uses on its mbarriers: one CTA waits on a barrier that nothing ever
+ * completes, gives up after `budget_cycles` SM clock cycles (1 .. 2^31), sets
+ * the device error word to TQ_ERR_TIMEOUT and exits, leaving the context
+ * usable.  Enqueued on `stream`; the status appears at the next
+ * tq_sync_check.  TQ_ERR_INVALID_ARG for a budget outside the range.
+ */
+tq_status tq_check_wait_expiry(int64_t budget_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

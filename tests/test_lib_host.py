@@ -93,6 +93,12 @@ def test_params_validation():
     assert lib.tq_params_create(128, 3, 0x201, 0, 128, p, None, None, C.byref(h)) == 1  # unknown flag
 
 
+def test_wait_expiry_check_validates_budget():
+    lib = L.lib()
+    assert lib.tq_check_wait_expiry(0, None) == 1
+    assert lib.tq_check_wait_expiry((1 << 31) + 1, None) == 1
+
+
 def test_unbiased_mode_handle():
     # Q_MSE with the unbiased (EDEN) scale: same code geometry as Q_MSE, and
     # accepted by the Q_MSE entry points' validation (a Q_prod call is not)

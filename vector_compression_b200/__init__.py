@@ -317,6 +317,11 @@ def tq_decode_step(kp: TQParams, vp: TQParams, q, k_new, v_new, kcache, vcache, 
     return out
 
 
+def tq_check_wait_expiry(budget_cycles: int, stream=None):
+    """Run the bounded-wait expiry path once (the status shows at tq_sync_check)."""
+    L.check("tq_check_wait_expiry", L.lib().tq_check_wait_expiry(int(budget_cycles), _stream(stream)))
+
+
 def tq_sync_check(stream=None):
     """Synchronize and raise if a kernel flagged a device-side error."""
     L.check("tq_sync_check", L.lib().tq_sync_check(_stream(stream)))

@@ -47,6 +47,7 @@ SIGNATURES = {
     "tq_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64, _i64, _f,
                             _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "tq_sync_check": (_i, [_vp]),
+    "tq_check_wait_expiry": (_i, [C.c_int64, _vp]),
 }
 
 

@@ -40,6 +40,36 @@ unsigned* device_error_ptr() {
   return ptrs[dev];
 }
 
+// One CTA waits on an mbarrier that nothing arrives at, with the kernels'
+// bounded-wait structure (try_wait polling against a clock64 budget), and
+// records the expiry in the error word.
+__global__ void wait_expiry_kernel(long long budget, unsigned* err) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = (uint32_t)__cvta_generic_to_shared(&bar);
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const long long t0 = clock64();
+    while (true) {
+      uint32_t done;
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}\n"
+          : "=r"(done)
+          : "r"(b), "r"(0u)
+          : "memory");
+      if (done) break;  // cannot happen: phase 0 needs one arrival
+      if (clock64() - t0 > budget) {
+        atomicCAS(err, 0u, (unsigned)TQ_ERR_TIMEOUT);
+        break;
+      }
+    }
+  }
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -656,6 +686,14 @@ tq_status tq_decode_attention(const tq_params* kp, const tq_params* vp, const fl
   return cuda_status(tq::launch_decode_attention(kp->q, vp->q, q, L, B, Hq, Hkv, seq, cap, scale,
                                                  kcodes, ksigns, knorms, krnorms, vcodes, vnorms,
                                                  out, ws, stream));
+}
+
+tq_status tq_check_wait_expiry(int64_t budget_cycles, void* stream) {
+  if (budget_cycles < 1 || budget_cycles > (int64_t(1) << 31)) return TQ_ERR_INVALID_ARG;
+  unsigned* err = tq::device_error_ptr();
+  if (!err) return TQ_ERR_CUDA;
+  tq::wait_expiry_kernel<<<1, 32, 0, tq::S(stream)>>>((long long)budget_cycles, err);
+  return cudaGetLastError() == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }
 
 tq_status tq_sync_check(void* stream) {
