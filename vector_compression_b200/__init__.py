@@ -20,8 +20,10 @@ from ._lib import (BF16, F16, F32, LAYOUT_BLOCK32, LAYOUT_ROW, MODE_MSE, MODE_MS
 __all__ = [
     "TQParams", "tq_build_codebook", "tq_make_rotation", "tq_params_create", "tq_encode_mse", "tq_encode_prod",
     "tq_decode", "tq_scores", "tq_decode_attention", "tq_decode_attention_workspace_size",
-    "tq_decode_attention_noalloc",
-    "tq_sync_check", "tq_version", "lib_path", "TQError",
+    "tq_decode_attention_noalloc", "tq_decode_step", "tq_decode_step_workspace_size",
+    "tq_check_wait_expiry", "tq_sync_check", "tq_version", "lib_path", "TQError",
+    "F32", "F16", "BF16", "LAYOUT_ROW", "LAYOUT_BLOCK32", "MODE_MSE", "MODE_PROD", "MODE_MSE_UNBIASED",
+    "STORE_RNORM_F16", "ROT_HADAMARD", "ROT_DENSE",
 ]
 
 
