@@ -250,11 +250,13 @@ tq_status tq_scores_workspace_size(const tq_params* kp, int64_t nq, int64_t n_ve
  * Pattern 1: scores from compressed keys, softmax, weighted sum of the
  * Q_MSE-reconstructed values), fused: the values are averaged in the rotated
  * domain and Pi_V^T is applied once per output (Pi^T is linear).
- *   kp      Q_prod handle of the keys; vp Q_MSE handle of the values; both
- *           with the same d.
+ *   kp      Q_prod handle of the keys; vp Q_MSE handle of the values
+ *           (TQ_MODE_MSE or TQ_MODE_MSE_UNBIASED); both with the same d and
+ *           rotation kind.
  *   q       DEVICE float [L][B][Hq][d] (one query token per head)
  *   Hq, Hkv query / KV heads, Hq a multiple of Hkv; query head h reads KV
- *           head h / (Hq / Hkv).
+ *           head h / (Hq / Hkv); at most 16 query heads per KV head
+ *           (TQ_ERR_UNSUPPORTED above).
  *   seq     valid tokens per (layer, batch, kv-head), >= 1
  *   cap     token slots per (layer, batch, kv-head) in the cache, >= seq, a
  *           multiple of 32
