@@ -25,8 +25,9 @@
 // and sums are exact integers; the only rounding is the fixed point itself
 // (2^-24 of the largest query entry, 2^-16 of the largest weight).
 //
-// Per CTA: one (layer, batch, kv-head) group and one chunk, 4 warps, in
-// sub-chunks of up to 512 tokens whose keys, value blocks and norms are
+// Per CTA: one (layer, batch, kv-head) group and one chunk, d_pad / 32 warps
+// (4 at d_pad 128, 8 at 256), in sub-chunks of up to 384 (d_pad 128) or 192
+// (d_pad 256) tokens whose keys, value blocks and norms are
 // staged in shared memory by bulk asynchronous copies (the next sub-chunk's
 // keys load while this one's weights and values are formed, its values while
 // the next scores are):
@@ -53,11 +54,8 @@ namespace attn3 {
 
 using attn2::Params;
 
-constexpr int kWarps = 4;
-constexpr int kThreads = 32 * kWarps;
-constexpr int DP = 128;            // rotated dimension
-constexpr int WPP = DP / 32;       // words per code plane
-constexpr int SC = 384;            // tokens per sub-chunk (a multiple of 64)
+// The geometry (warps, words per plane, sub-chunk length) follows d_pad:
+// see Layout.
 constexpr float kQMax = 8323072.0f;  // 127 * 2^16: the hi byte stays in [-127, 127]
 
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

@@ -20,11 +20,13 @@
 // TMEM buffer g and every second tile; one thread per vector computes
 // n = ||u|| / sqrt(d_pad) and the bit planes (sign plane and thermometer
 // planes of |u| against the positive boundaries scaled by ||u||).
-// Q_prod (encode_prod_kernel): one group of 16 warps, four threads per vector
-// (32 columns each); the epilogue writes r = u / ||u|| - C[idx] (times 2^10,
+// Q_prod (encode_prod_rows_kernel, the default): the same two groups and one
+// thread per vector; the epilogue writes r = u / ||u|| - C[idx] (times 2^10,
 // split into fp16 hi + lo parts) back over u, a second MMA forms S r (A = r
-// from TMEM, B = S from shared memory) while the next tile is quantized, and
-// the epilogue then reads its rows of S r for the QJL sign words.
+// from TMEM, B = S from shared memory), and the group packs the QJL sign
+// words of its rows while the other group quantizes the next tile.  The
+// earlier form (encode_prod_kernel: one group, two or four threads per
+// vector, signs read one tile later) is kept for cross-checks.
 // Exact boundary ties on the negative side resolve toward zero here (the
 // oracle resolves them to the lower cell); such values lie inside the parity
 // window by definition.
