@@ -321,6 +321,62 @@ def test_qprod_unbiased_over_seeds_of_S():
     assert est.var() <= bound * 1.05
 
 
+def _fp16_gaussian(rng, shape):
+    # the library's S: standard normal draws rounded to the nearest IEEE
+    # binary16 value (round to nearest even), held exactly in fp32
+    return rng.standard_normal(shape).astype(np.float16).astype(np.float32)
+
+
+def test_half_gaussian_identity_fp16_rounded_draws():
+    # The identity behind the QJL estimator (§8) with the rows of S that the
+    # library accepts: N(0, 1) entries rounded to fp16.  Rounding moves each
+    # entry by at most 2^-11 of its value, far inside the Monte Carlo error
+    # at 4e5 draws, so the identity must still hold within 4 standard errors.
+    rng = np.random.default_rng(8)
+    d = 16
+    x = rng.standard_normal(d)
+    y = rng.standard_normal(d)
+    S = _fp16_gaussian(rng, (400_000, d)).astype(np.float64)
+    v = (S @ y) * np.where(S @ x >= 0, 1.0, -1.0)
+    want = math.sqrt(2 / math.pi) * x @ y / np.linalg.norm(x)
+    assert abs(v.mean() - want) < 4 * v.std() / math.sqrt(len(v))
+    # the second moment that the variance bound uses is unchanged too:
+    # E[(s.y)^2] = ||y||^2 within 4 standard errors
+    w = (S @ y) ** 2
+    assert abs(w.mean() - y @ y) < 4 * w.std() / math.sqrt(len(w))
+
+
+def test_qprod_unbiased_over_seeds_of_fp16_S():
+    # [NOTES] eq. (3) / Q_prod with the fp16-rounded Gaussian S the library
+    # requires: for fixed x, q, Pi the estimator averaged over 12,000
+    # independent fp16-rounded draws of S equals <q, x> within 3 standard
+    # errors, and its variance obeys the QJL bound pi/(2m) ||r||^2 ||q'||^2 n^2
+    # (explainer §8, Lemma 4 and the half-Gaussian identity).
+    rng = np.random.default_rng(22)
+    d, m, bits = 32, 32, 3
+    x = rng.standard_normal(d) * 2.0
+    qv = rng.standard_normal(d)
+    base = _draws(d, m, 1, f64=True)
+    q0 = o.Quantizer(d, bits, prod=True, draws=base)
+    n, y = q0.rotate_unit(x[None])
+    r = y - q0.centroids[q0.quantize(y)]
+    est = []
+    for s in range(12000):
+        dr = dict(base)
+        dr["S"] = _fp16_gaussian(np.random.default_rng([22, s]), (m, d))
+        assert np.array_equal(dr["S"], dr["S"].astype(np.float16).astype(np.float32))
+        q = o.Quantizer(d, bits, prod=True, draws=dr)
+        e = q.encode(x[None])
+        est.append(q.scores(qv[None], e["idx"], e["norms"], e["signs"], e["rnorms"])[0, 0])
+    est = np.array(est)
+    truth = qv @ x
+    se = est.std() / math.sqrt(len(est))
+    assert abs(est.mean() - truth) < 3 * se
+    qp = q0.rot.apply(qv)
+    bound = math.pi / (2 * m) * float(r[0] @ r[0]) * float(qp @ qp) * float(n[0] ** 2)
+    assert est.var() <= bound * 1.05
+
+
 def test_qmse_shrinkage_over_haar_rotations():
     # §7: with a uniformly random rotation, E<y, x~> = lambda_b <y, x>, with
     # lambda_b = d sum_i c_i^2 P_i from the codebook (within 3 standard errors).
