@@ -294,13 +294,16 @@ tq_status tq_decode_attention_workspace_size(const tq_params* kp, const tq_param
  * until the process exits.  A call whose tq_decode_attention_workspace_size
  * is larger returns TQ_ERR_WORKSPACE and enqueues nothing.
  *
- * The first call on each device looks up the array's device address (with
- * that device current) and caches it; make that first call before any
- * stream capture.  Every call shares the same array.  The attention kernels
- * overwrite every scratch byte they read, so nothing relies on its previous
- * contents; but calls that overlap on the GPU (other streams, other host
- * threads) race on the array and corrupt each other's results -- serialize
- * them.
+ * Every call looks up the array's device address in the caller's current
+ * device and context (nothing is cached, so the address stays right after
+ * cudaDeviceReset or when the caller switches contexts).  The first call in
+ * a context may load the library's module into it: make that first call
+ * before any stream capture.  Every call shares the same array.  The
+ * attention kernels write every scratch byte they later read within the
+ * same call (a chunk whose staging wait expires writes an empty partial),
+ * so nothing relies on the array's previous contents; but calls that
+ * overlap on the GPU (other streams, other host threads) race on the array
+ * and corrupt each other's results -- serialize them.
  *
  * Arguments, layouts, results and the other errors are those of
  * tq_decode_attention.
@@ -346,16 +349,19 @@ tq_status tq_decode_step_workspace_size(const tq_params* kp, const tq_params* vp
 /*
  * tq_sync_check -- synchronize `stream` and report (then clear) the device
  * error word that kernels set when a bounded wait expires (TQ_ERR_TIMEOUT)
- * or an internal check fails (TQ_ERR_INTERNAL).
+ * or an internal check fails (TQ_ERR_INTERNAL).  When it reports
+ * TQ_ERR_TIMEOUT, the outputs of the calls enqueued since the previous check
+ * are not valid results: a kernel whose wait expired skipped the rest of its
+ * work (an attention chunk then contributes nothing to its heads' outputs).
  */
 tq_status tq_sync_check(void* stream);
 
 /*
- * tq_check_wait_expiry -- exercise the bounded-wait path that every kernel
- * uses on its mbarriers: one CTA waits on a barrier that nothing ever
- * completes, gives up after `budget_cycles` SM clock cycles (1 .. 2^31), sets
- * the device error word to TQ_ERR_TIMEOUT and exits, leaving the context
- * usable.  Enqueued on `stream`; the status appears at the next
+ * tq_check_wait_expiry -- exercise the bounded-wait helper that every kernel
+ * uses on its mbarriers, in both of its forms (polling and suspending): one
+ * CTA waits on barriers that nothing ever completes, gives up after
+ * `budget_cycles` SM clock cycles (1 .. 2^31) per wait, sets the device error
+ * word to TQ_ERR_TIMEOUT and exits, leaving the context usable.  Enqueued on `stream`; the status appears at the next
  * tq_sync_check.  TQ_ERR_INVALID_ARG for a budget outside the range.
  */
 tq_status tq_check_wait_expiry(int64_t budget_cycles, void* stream);

@@ -141,4 +141,3 @@ def test_encode_and_attention_validation_before_launch():
     assert lib.tq_decode_attention(h, h, fake, 1, 1, 8, 2, 64, 64, f, *args, None, 0, None) == 1
     sz = C.c_size_t()
     assert lib.tq_decode_attention_workspace_size(h, h, 1, 1, 7, 2, 64, C.byref(sz)) == 1  # Hq % Hkv
-    assert lib.tq_decode_workspace_size if hasattr(lib, "tq_decode_workspace_size") else True

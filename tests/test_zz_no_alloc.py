@@ -65,6 +65,20 @@ def test_noalloc_matches_workspace_entry_point_twice():
     tq.tq_sync_check()
 
 
+def test_noalloc_python_wrapper_matches_workspace_entry_point():
+    # the binding's wrapper (which makes q's device current around the call)
+    kp, vp, q, kc, vc, dims = _case(14, 500, 512, 4)
+    scale = 1 / math.sqrt(128)
+    got = tq.tq_decode_attention_noalloc(kp, vp, q, kc, vc, 500, 512, scale)
+    want = tq.tq_decode_attention(kp, vp, q, kc, vc, 500, 512, scale)
+    torch.cuda.synchronize()
+    g, w = got.cpu().numpy(), want.cpu().numpy()
+    assert np.all(np.isfinite(g))
+    err = np.linalg.norm(g - w, axis=-1) / np.linalg.norm(w, axis=-1)
+    assert err.max() <= REL_TOL, err.max()
+    tq.tq_sync_check()
+
+
 def test_noalloc_rejects_oversized_requests():
     kp, vp, q, kc, vc, dims = _case(13, 64, 64, 4)
     need = tq.tq_decode_attention_workspace_size(kp, vp, 4096, 64, 32, 8, 32768)

@@ -278,10 +278,12 @@ def tq_decode_attention_noalloc(kp: TQParams, vp: TQParams, q, kcache, vcache, s
     if out is None:
         out = torch.empty((Ln, B, Hq, d), dtype=torch.float32, device=q.device)
     qc = q.contiguous()
-    L.check("tq_decode_attention_noalloc", L.lib().tq_decode_attention_noalloc(
-        kp.handle, vp.handle, _ptr(qc), Ln, B, Hq, Hkv, seq, cap, float(scale),
-        _ptr(kcodes), _ptr(ksigns), _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms),
-        _ptr(out), _stream(stream)))
+    # the scratch array used is the current device's: make q's device current
+    with torch.cuda.device(q.device):
+        L.check("tq_decode_attention_noalloc", L.lib().tq_decode_attention_noalloc(
+            kp.handle, vp.handle, _ptr(qc), Ln, B, Hq, Hkv, seq, cap, float(scale),
+            _ptr(kcodes), _ptr(ksigns), _ptr(knorms), _ptr(krnorms), _ptr(vcodes), _ptr(vnorms),
+            _ptr(out), _stream(stream)))
     return out
 
 

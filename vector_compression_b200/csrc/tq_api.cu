@@ -4,12 +4,11 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
-#include <cstdio>
-#include <cstdlib>
 
 #include "tq_attention.cuh"
-#include "tq_attn2.h"
+#include "tq_attn_params.h"
 #include "tq_attn3.h"
 #include "tq_device.cuh"
 #include "tq_encode.cuh"
@@ -19,6 +18,7 @@
 #include "tq_gemm.cuh"
 #include "tq_internal.h"
 #include "tq_scores.cuh"
+#include "tq_wait.cuh"
 
 namespace tq {
 
@@ -28,46 +28,29 @@ __device__ unsigned int g_device_error = 0;
 
 namespace {
 
+// Address of the error word in the current context, looked up on every call
+// (a cached address would go stale after cudaDeviceReset or a context switch).
 unsigned* device_error_ptr() {
-  static unsigned* ptrs[128] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 128) return nullptr;
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) ptrs[dev] = (unsigned*)p;
-  }
-  return ptrs[dev];
+  void* p = nullptr;
+  return cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess ? (unsigned*)p : nullptr;
 }
 
-// One CTA waits on an mbarrier that nothing arrives at, with the kernels'
-// bounded-wait structure (try_wait polling against a clock64 budget), and
-// records the expiry in the error word.
+// One CTA waits, with the kernels' bounded-wait helper in both of its forms
+// (polling test_wait, suspending try_wait), on mbarriers that nothing
+// arrives at; each expiry is recorded in the error word.
 __global__ void wait_expiry_kernel(long long budget, unsigned* err) {
-  __shared__ __align__(8) uint64_t bar;
-  const uint32_t b = (uint32_t)__cvta_generic_to_shared(&bar);
+  __shared__ __align__(8) uint64_t bar[2];
+  const uint32_t b0 = (uint32_t)__cvta_generic_to_shared(&bar[0]);
+  const uint32_t b1 = (uint32_t)__cvta_generic_to_shared(&bar[1]);
   if (threadIdx.x == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b0));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b1));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    const long long t0 = clock64();
-    while (true) {
-      uint32_t done;
-      asm volatile(
-          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-          "selp.u32 %0, 1, 0, p;\n\t}\n"
-          : "=r"(done)
-          : "r"(b), "r"(0u)
-          : "memory");
-      if (done) break;  // cannot happen: phase 0 needs one arrival
-      if (clock64() - t0 > budget) {
-        atomicCAS(err, 0u, (unsigned)TQ_ERR_TIMEOUT);
-        break;
-      }
-    }
-  }
+  // phase 0 of each needs one arrival, which never comes
+  if (threadIdx.x == 0) bounded_wait<false>(b0, 0u, err, budget);
+  if (threadIdx.x == 1) bounded_wait<true>(b1, 0u, err, budget);
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -76,14 +59,20 @@ inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline size_t dtype_size(int dt) { return dt == TQ_F32 ? 4 : 2; }
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// SM count of the current device, cached per device ordinal (a device's SM
+// count does not change; the cache entries are written once, atomically).
 int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cache[kMaxDev];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < kMaxDev) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
   }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev >= 0 && dev < kMaxDev) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -231,18 +220,8 @@ size_t encode_workspace_bytes(const QParams& qp, bool prod, int64_t n_vec) {
 }  // namespace
 
 // Encoder selection: the tensor-core encoder whenever it covers a request,
-// else the thread-per-vector one, else the warp-per-vector kernels.  The
-// environment variable TQ_ENCODE_V2=1 skips the first, TQ_ENCODE_V1=1 both
-// (the older kernels stay as second implementations for cross-checks).
-static const bool g_encode_v2 = [] {
-  const char* e = getenv("TQ_ENCODE_V1");
-  return !(e && e[0] == '1');
-}();
-static const bool g_encode_tc = [] {
-  const char* e = getenv("TQ_ENCODE_V2");
-  return g_encode_v2 && !(e && e[0] == '1');
-}();
-
+// else the thread-per-vector one (f32 rows, d_pad 256), else the
+// warp-per-vector kernels (any other shape).
 int launch_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_vec, int64_t ld,
                   int64_t seg_len, int64_t seg_cap, int layout, uint32_t* codes, uint32_t* signs,
                   float* norms, float* rnorms, void* ws, void* stream) {
@@ -250,10 +229,10 @@ int launch_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n
   cudaStream_t st = S(stream);
   {
     cudaError_t e2;
-    if (g_encode_tc && enc3::try_encode(qp, prod, x, dt, n_vec, ld, seg_len, seg_cap, layout, codes,
+    if (enc3::try_encode(qp, prod, x, dt, n_vec, ld, seg_len, seg_cap, layout, codes,
                                         signs, norms, rnorms, device_error_ptr(), num_sms(), st, &e2))
       return e2;
-    if (g_encode_v2 && try_encode_v2(qp, prod, x, dt, n_vec, ld, seg_len, seg_cap, layout, codes,
+    if (try_encode_v2(qp, prod, x, dt, n_vec, ld, seg_len, seg_cap, layout, codes,
                                      signs, norms, rnorms, st, &e2))
       return e2;
   }
@@ -346,11 +325,9 @@ int launch_scores(const QParams& qp, const float* qrot, const float* u, int64_t 
   if (nq == 0 || n_vec == 0) return cudaSuccess;
   const int qt = score_query_tile(qp);
   const size_t smem = (size_t)qt * (qp.d_pad + qp.m) * sizeof(float);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
-    attr_set = true;
-  }
+  // function attributes are per device: set on every call (a cheap host call)
+  cudaError_t ae = cudaFuncSetAttribute(scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
+  if (ae != cudaSuccess) return ae;
   dim3 grid((unsigned)ceil_div(n_vec, kScoreThreads), (unsigned)ceil_div(nq, qt));
   scores_kernel<<<grid, kScoreThreads, smem, S(stream)>>>(qp, qrot, u, nq, qt, codes, signs, norms,
                                                           rnorms, n_vec, scores);
@@ -389,26 +366,18 @@ size_t attention_workspace(const QParams& kp, const QParams& vp, int L, int B, i
   return bytes;
 }
 
-// The tensor-core kernels (int8: tq_attn3.cu, fp16: tq_attn2.cu) cover
-// at most 8 query heads per KV head and key codes of 1..3 bits: the int8
-// kernel d_pad = 128 with m = 64 or 128 and d_pad = 256 with m = 256, the
-// fp16 kernel d_pad = 128 with m = 128.  The int8 kernel runs unless
-// TQ_ATTN_V2=1 selects the fp16 one, and TQ_ATTN_V1=1 selects the SIMT kernel
-// for every shape.
-static const bool g_attn_v2 = [] {
-  const char* e = getenv("TQ_ATTN_V1");
-  return !(e && e[0] == '1');
-}();
-static const bool g_attn_v3 = [] {
-  const char* e = getenv("TQ_ATTN_V2");
-  return g_attn_v2 && !(e && e[0] == '1');
-}();
-
-static bool attn2_covers(const QParams& kp, const QParams& vp, int G) {
-  const bool shape = (kp.d_pad == 128 && vp.d_pad == 128 && (kp.m == 128 || (kp.m == 64 && g_attn_v3))) ||
-                     (kp.d_pad == 256 && vp.d_pad == 256 && kp.m == 256 && g_attn_v3);
-  return g_attn_v2 && kp.rot == TQ_ROT_HADAMARD && shape && G >= 1 && G <= 8 && kp.k >= 1 && kp.k <= 3 &&
-         vp.k >= 1 && vp.k <= 4;
+// The int8 tensor-core kernel (tq_attn3.cu) covers at most 8 query heads per
+// KV head, key codes of 1..3 bits and value codes of 1..4 bits at d_pad = 128
+// with m = 64 or 128 and at d_pad = 256 with m = 256, with the norm and sign
+// arrays 16-byte aligned (it stages them with bulk copies); the SIMT kernel
+// (tq_attention.cuh) covers every other shape.
+static bool attn3_covers(const QParams& kp, const QParams& vp, int G, const void* ksigns,
+                         const void* knorms, const void* krnorms, const void* vnorms) {
+  const bool shape = (kp.d_pad == 128 && vp.d_pad == 128 && (kp.m == 128 || kp.m == 64)) ||
+                     (kp.d_pad == 256 && vp.d_pad == 256 && kp.m == 256);
+  return kp.rot == TQ_ROT_HADAMARD && shape && G >= 1 && G <= 8 && kp.k >= 1 && kp.k <= 3 &&
+         vp.k >= 1 && vp.k <= 4 && aligned16(ksigns) && aligned16(knorms) && aligned16(krnorms) &&
+         aligned16(vnorms);
 }
 
 int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q, int L, int B,
@@ -436,8 +405,8 @@ int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q
   sh.seq = seq;
   sh.cap = cap;
   sh.scale = scale;
-  if (attn2_covers(kp, vp, sh.G)) {
-    attn2::Params p2;
+  if (attn3_covers(kp, vp, sh.G, ksigns, knorms, krnorms, vnorms)) {
+    attn::Params p2;
     p2.G = sh.G;
     p2.chunk = chunk;
     p2.n_chunks = n_chunks;
@@ -456,26 +425,17 @@ int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q
     p2.vnorms = vnorms;
     p2.part = part;
     p2.err = device_error_ptr();
-    attn2::odd_feature_coefs(kp.centroids, kp.k, p2.kalpha, &p2.kalpha_sum);
-    attn2::odd_feature_coefs(vp.centroids, vp.k, p2.valpha, &p2.valpha_sum);
+    attn::odd_feature_coefs(kp.centroids, kp.k, p2.kalpha, &p2.kalpha_sum);
+    attn::odd_feature_coefs(vp.centroids, vp.k, p2.valpha, &p2.valpha_sum);
     const dim3 grid((unsigned)n_chunks, (unsigned)sh.groups);
-    // the int8 kernel stages rows with bulk copies: 16-byte aligned arrays
-    const bool v3 = g_attn_v3 && aligned16(ksigns) && aligned16(knorms) && aligned16(krnorms) &&
-                    aligned16(vnorms);
-    cudaError_t ce = cudaErrorInvalidValue;
-    if (v3)
-      ce = attn3::launch(p2, kp.k, vp.k, kp.m, kp.d_pad, grid, st);
-    else if (kp.m == 128 && kp.d_pad == 128)
-      ce = attn2::launch(p2, kp.k, vp.k, grid, st);
+    const cudaError_t ce = attn3::launch(p2, kp.k, vp.k, kp.m, kp.d_pad, grid, st);
     if (ce != cudaSuccess) return ce;
   } else {
   const size_t smem = (size_t)sh.G * (kp.d_pad + kp.m) * sizeof(float);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(attention_chunk_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-    cudaFuncSetAttribute(attention_chunk_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
-    attr_set = true;
-  }
+  // function attributes are per device: set on every call (a cheap host call)
+  cudaError_t ae = cudaFuncSetAttribute(kp.d_pad <= 128 ? attention_chunk_kernel<1> : attention_chunk_kernel<2>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+  if (ae != cudaSuccess) return ae;
   dim3 grid((unsigned)n_chunks, (unsigned)sh.groups);
   if (kp.d_pad <= 128)
     attention_chunk_kernel<1><<<grid, kAttnThreads, smem, st>>>(kp, vp, sh, qrot, u, kcodes, ksigns, knorms, krnorms, vcodes, vnorms, part);
@@ -519,16 +479,7 @@ int read_and_clear_device_error(void* stream, unsigned* err) {
 
 namespace {
 
-// With TQ_VERBOSE=1 in the environment, CUDA failures are also named on stderr.
-tq_status cuda_status(int e) {
-  if (e == cudaSuccess) return TQ_OK;
-  static const bool verbose = [] {
-    const char* v = getenv("TQ_VERBOSE");
-    return v && v[0] == '1';
-  }();
-  if (verbose) fprintf(stderr, "libtq: CUDA error %d (%s)\n", e, cudaGetErrorName((cudaError_t)e));
-  return TQ_ERR_CUDA;
-}
+tq_status cuda_status(int e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
 
 tq_status check_segments(int64_t n_vec, int64_t* seg_len, int64_t* seg_cap, bool block) {
   if (n_vec < 0) return TQ_ERR_INVALID_ARG;

@@ -3,7 +3,7 @@
 // weighted sum of the Q_MSE-reconstructed values; TurboQuant blog notes,
 // Q_prod estimator; explainer §8).
 //
-// Exact bit features, as in the fp16 kernel (tq_attn2.cu): a symmetric
+// Exact bit features: a symmetric
 // codebook is an odd function of the index bits, C[idx] = sum over odd subsets
 // S of alpha_S (2 b_S - 1), b_S the XOR of the bits in S, so every
 // contraction is against 0/1 bit matrices:
@@ -45,14 +45,15 @@
 
 #include <cstdint>
 
-#include "tq_attn2.h"
+#include "tq_attn_params.h"
 #include "tq_attn3.h"
 #include "tq_device.cuh"
+#include "tq_wait.cuh"
 
 namespace tq {
 namespace attn3 {
 
-using attn2::Params;
+using attn::Params;
 
 // The geometry (warps, words per plane, sub-chunk length) follows d_pad:
 // see Layout.
@@ -154,24 +155,11 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 __device__ __forceinline__ void mbar_expect(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
-// Bounded wait for the phase with the given parity (suspend-hinted); false
-// and the device error word set if it does not complete within ~2^31 cycles.
+// Bounded wait for the phase with the given parity: false, and the device
+// error word set (when err is not null), if it does not complete within the
+// wait budget.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
-  const long long t0 = clock64();
-  while (true) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(done)
-        : "r"(bar), "r"(parity), "r"(20000u)
-        : "memory");
-    if (done) return true;
-    if (clock64() - t0 > (1LL << 31)) {
-      if (err) atomicCAS(err, 0u, (unsigned)TQ_ERR_TIMEOUT);
-      return false;
-    }
-  }
+  return bounded_wait<true>(bar, parity, err);
 }
 
 template <int KK, int KV, int NT, int MQ, int DPT>
@@ -615,10 +603,17 @@ __global__ void __launch_bounds__(DPT) attn_kernel(Params P) {
     __syncthreads();
   }
   if (!ok) {
-    // a staging wait expired (error word set): let copies still in flight land
+    // a staging wait expired (error word set): let copies still in flight
+    // land, and leave an empty partial (m = -inf: the combine skips it) so
+    // that nothing downstream reads stale workspace
     if (tid == 0) {
       mbar_wait(bk, phase, nullptr);
       mbar_wait(bv, phase, nullptr);
+    }
+    if (tid < G) {
+      float* pp = P.part + (((int64_t)grp * P.n_chunks + chunk) * G + tid) * (int64_t)(DP + 2);
+      pp[0] = -INFINITY;
+      pp[1] = 0.f;
     }
     return;
   }

@@ -1,4 +1,6 @@
-// Tensor-core decode attention (tq_attn2.cu): launch parameters.
+// Launch parameters shared by the tensor-core decode-attention kernels
+// (tq_attn3.cu, tq_attn4.cu) and the odd-subset coefficients of a symmetric
+// codebook that both use.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -6,7 +8,7 @@
 #include <cstdint>
 
 namespace tq {
-namespace attn2 {
+namespace attn {
 
 struct Params {
   int G;          // query heads per KV head (1..8)
@@ -14,8 +16,8 @@ struct Params {
   int n_chunks;
   int64_t seq, cap;
   float scale, kappa;
-  const float* qrot;  // [groups * G][128]
-  const float* u;     // [groups * G][128]
+  const float* qrot;  // [groups * G][d_pad]
+  const float* u;     // [groups * G][m]
   const uint32_t* kcodes;
   const uint32_t* ksigns;
   const float* knorms;
@@ -24,7 +26,7 @@ struct Params {
   const uint32_t* vcodes;
   const float* vnorms;
   float* part;
-  unsigned* err;    // device error word (bounded waits of the int8 kernel)
+  unsigned* err;    // device error word (bounded waits)
   float kalpha[8];  // odd-subset coefficients of the key codebook
   float kalpha_sum;
   float valpha[8];  // and of the value codebook
@@ -36,7 +38,5 @@ struct Params {
 // then the triples ({0,1,2}; for k = 4 also {0,1,3}, {0,2,3}, {1,2,3}).
 void odd_feature_coefs(const float* centroids, int k, float* alpha, float* alpha_sum);
 
-cudaError_t launch(const Params& p, int kk, int kv, dim3 grid, cudaStream_t st);
-
-}  // namespace attn2
+}  // namespace attn
 }  // namespace tq

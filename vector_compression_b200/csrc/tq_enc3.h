@@ -62,11 +62,6 @@ inline uint32_t smem_bytes(int mode, int m) {
   return kRotBytes + (mode == MODE_PROD ? (uint32_t)m * kDP * 2 : 0u) + kStages * kTileBytes + 1024;
 }
 
-// Threads per vector of the Q_prod encoder: 1 (two epilogue groups on
-// alternate tiles), or 2 / 4 (one group per tile) with TQ_PROD_TPR=2 / 4 in
-// the environment.
-int prod_tpr();
-
 cudaError_t launch_f16(int mode, const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,
                        cudaStream_t st);
 cudaError_t launch_bf16(int mode, const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,

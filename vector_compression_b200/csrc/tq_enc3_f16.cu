@@ -11,22 +11,10 @@ cudaError_t launch_one(const CUtensorMap& map, const QParams& qp, const Args& a,
                        cudaStream_t st) {
   const int smem = (int)smem_bytes(MODE, qp.m);
   if constexpr (MODE == MODE_PROD) {
-    if (prod_tpr() == 1) {
-      auto kern = encode_prod_rows_kernel<__half, K>;
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return e;
-      kern<<<ctas, kThreads, smem, st>>>(map, qp, a);
-    } else if (prod_tpr() == 2) {
-      auto kern = encode_prod_kernel<__half, K, 2>;
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return e;
-      kern<<<ctas, prod_threads<2>(), smem, st>>>(map, qp, a);
-    } else {
-      auto kern = encode_prod_kernel<__half, K, 4>;
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return e;
-      kern<<<ctas, prod_threads<4>(), smem, st>>>(map, qp, a);
-    }
+    auto kern = encode_prod_rows_kernel<__half, K>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, kThreads, smem, st>>>(map, qp, a);
   } else {
     auto kern = encode_tc_kernel<__half, K, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

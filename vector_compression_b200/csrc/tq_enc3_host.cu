@@ -2,7 +2,6 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
-#include <cstdlib>
 #include <mutex>
 
 #include "tq_enc3.h"
@@ -26,14 +25,6 @@ PFN_cuTensorMapEncodeTiled encode_tiled_fn() {
 }
 
 }  // namespace
-
-int prod_tpr() {
-  static const int tpr = [] {
-    const char* e = getenv("TQ_PROD_TPR");
-    return (e && e[0] == '4') ? 4 : (e && e[0] == '2') ? 2 : 1;
-  }();
-  return tpr;
-}
 
 bool try_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_vec, int64_t ld,
                 int64_t seg_len, int64_t seg_cap, int layout, uint32_t* codes, uint32_t* signs,

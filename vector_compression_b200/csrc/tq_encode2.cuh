@@ -31,6 +31,7 @@
 #pragma once
 
 #include "tq_device.cuh"
+#include "tq_wait.cuh"
 
 namespace tq {
 namespace enc2 {
@@ -327,24 +328,10 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Bounded wait for the mbarrier phase with the given parity.  Returns false
-// (and sets the device error word) if it does not complete in ~2^31 cycles.
+// Bounded wait for the mbarrier phase with the given parity: false, and the
+// device error word set, if it does not complete within the wait budget.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
-  const long long t0 = clock64();
-  while (true) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if (clock64() - t0 > (1LL << 31)) {
-      atomicCAS(err, 0u, (unsigned)TQ_ERR_TIMEOUT);
-      return false;
-    }
-  }
+  return bounded_wait<true>(bar, parity, err);
 }
 
 // ------------------------------------------------------------------ kernel

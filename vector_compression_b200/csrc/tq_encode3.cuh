@@ -20,13 +20,11 @@
 // TMEM buffer g and every second tile; one thread per vector computes
 // n = ||u|| / sqrt(d_pad) and the bit planes (sign plane and thermometer
 // planes of |u| against the positive boundaries scaled by ||u||).
-// Q_prod (encode_prod_rows_kernel, the default): the same two groups and one
-// thread per vector; the epilogue writes r = u / ||u|| - C[idx] (times 2^10,
-// split into fp16 hi + lo parts) back over u, a second MMA forms S r (A = r
-// from TMEM, B = S from shared memory), and the group packs the QJL sign
-// words of its rows while the other group quantizes the next tile.  The
-// earlier form (encode_prod_kernel: one group, two or four threads per
-// vector, signs read one tile later) is kept for cross-checks.
+// Q_prod (encode_prod_rows_kernel): the same two groups and one thread per
+// vector; the epilogue writes r = u / ||u|| - C[idx] (times 2^10, split into
+// fp16 hi + lo parts) back over u, a second MMA forms S r (A = r from TMEM,
+// B = S from shared memory), and the group packs the QJL sign words of its
+// rows while the other group quantizes the next tile.
 // Exact boundary ties on the negative side resolve toward zero here (the
 // oracle resolves them to the lower cell); such values lie inside the parity
 // window by definition.
@@ -44,6 +42,7 @@
 
 #include "tq_device.cuh"
 #include "tq_enc3.h"
+#include "tq_wait.cuh"
 
 namespace tq {
 namespace enc3 {
@@ -65,30 +64,11 @@ __device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
                : "memory");
 }
 
-// One test of the phase with the given parity.
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t done;  // non-blocking test: polling measured faster than a suspending try_wait
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(done)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
-// Bounded wait for the phase with the given parity: false (and the device
-// error word set) if it has not completed within ~2^31 cycles.
+// Bounded wait for the phase with the given parity (non-blocking polls:
+// measured faster here than a suspending try_wait): false, and the device
+// error word set, if it has not completed within the wait budget.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
-  if (mbar_try(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try(bar, parity)) {
-    if (clock64() - t0 > (1LL << 31)) {
-      atomicCAS(err, 0u, (unsigned)TQ_ERR_TIMEOUT);
-      return false;
-    }
-  }
-  return true;
+  return bounded_wait<false>(bar, parity, err);
 }
 
 // Warp-uniform form: every lane waits, the warp proceeds only if all saw it.
@@ -676,339 +656,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-
-// ------------------------------------------------------------------ Q_prod kernel
-
-// Q_prod: one epilogue group of 4 TPR warps works on every tile; thread
-// (warp w, lane l) owns TMEM lane 32 (w % 4) + l (one vector) and the
-// 128 / TPR columns of column group (w - 2) / 4.  TMEM holds two tiles, each with a
-// 128-column slot for u (rewritten in place with the fp16 hi/lo residual, the
-// A operand of S r) and a 128-column slot for z = S r.  The S r MMA of tile L
-// runs while the epilogue quantizes tile L + 1; the signs of tile L are read
-// after that, so no warp waits for an MMA in steady state.
-template <int TPR>
-constexpr int prod_threads() { return 64 + 32 * 4 * TPR; }
-
-template <typename T, int K, int TPR>
-__global__ void __launch_bounds__(prod_threads<TPR>(), 1)
-    encode_prod_kernel(const __grid_constant__ CUtensorMap xmap, QParams qp, Args a) {
-  extern __shared__ unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages];
-  __shared__ __align__(8) uint64_t bar_accf[2], bar_aready[2], bar_zf[2], bar_zempty[2], bar_normx, bar_done;
-  __shared__ __align__(16) float ss_part[2][kRows][4];  // per tile parity: partial ||u||^2
-  __shared__ __align__(16) float rr_part[2][kRows][4];  // partial ||2^10 r||^2
-  __shared__ uint32_t tmem_base_s;
-  constexpr bool BF16 = !std::is_same<T, __half>::value;
-  constexpr int kEpiWarpsP = 4 * TPR;            // epilogue warps
-  constexpr int kThreadsP = prod_threads<TPR>();
-  constexpr int CPT = 4 / TPR;                   // 32-column chunks per thread
-  static_assert(TPR == 2 || TPR == 4, "two or four threads per vector");
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m = qp.m;
-  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  unsigned char* rot = smem;
-  unsigned char* smat = smem + kRotBytes;
-  unsigned char* stages = smat + m * kDP * 2;
-  constexpr uint32_t tmem_cols = 512u;
-
-  {
-    const uint16_t one = BF16 ? 0x3F80u : 0x3C00u;
-    for (int e = tid; e < kDP * (kDP / 8); e += kThreadsP) {
-      const int n = e / (kDP / 8), kc = e % (kDP / 8);
-      uint16_t v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int k = kc * 8 + i;
-        const uint32_t neg = (__popc(n & k) & 1) ^ ((qp.dmask[k >> 5] >> (k & 31)) & 1u);
-        v[i] = (uint16_t)(one | (neg << 15));
-      }
-      uint4 w;
-      w.x = v[0] | ((uint32_t)v[1] << 16);
-      w.y = v[2] | ((uint32_t)v[3] << 16);
-      w.z = v[4] | ((uint32_t)v[5] << 16);
-      w.w = v[6] | ((uint32_t)v[7] << 16);
-      *reinterpret_cast<uint4*>(rot + core_offset(n, kc * 8, kDP)) = w;
-    }
-    for (int e = tid; e < m * (kDP / 8); e += kThreadsP) {
-      const int row = e / (kDP / 8), kc = e % (kDP / 8);
-      const uint4 w = *reinterpret_cast<const uint4*>(qp.S16 + (size_t)row * kDP + kc * 8);
-      *reinterpret_cast<uint4*>(smat + core_offset(row, kc * 8, m)) = w;
-    }
-  }
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&bar_full[s]), 1);
-      mbar_init(smem_u32(&bar_empty[s]), 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&bar_accf[b]), 1);
-      mbar_init(smem_u32(&bar_aready[b]), 32 * kEpiWarpsP);  // every epilogue thread arrives
-      mbar_init(smem_u32(&bar_zf[b]), 1);
-      mbar_init(smem_u32(&bar_zempty[b]), 32 * kEpiWarpsP);
-    }
-    mbar_init(smem_u32(&bar_normx), 32 * kEpiWarpsP);
-    mbar_init(smem_u32(&bar_done), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&tmem_base_s)),
-                 "r"(tmem_cols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
-  }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base_s;
-  const int64_t G = gridDim.x;
-
-  if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      int issued = 0;
-      for (int L = 0;; ++L) {
-        const int64_t tile = blockIdx.x + (int64_t)L * G;
-        if (tile >= a.n_tiles) break;
-        const int s = L % kStages;
-        if (L >= kStages && !mbar_wait(smem_u32(&bar_empty[s]), ((L / kStages) - 1) & 1, a.err)) break;
-        const uint32_t dst = smem_u32(stages + s * kTileBytes);
-        mbar_arrive_tx(smem_u32(&bar_full[s]), kTileBytes);
-        tma_load_2d(dst, &xmap, 0, (int)(tile * kRows), smem_u32(&bar_full[s]));
-        tma_load_2d(dst + kTileBytes / 2, &xmap, 64, (int)(tile * kRows), smem_u32(&bar_full[s]));
-        issued = L + 1;
-      }
-      for (int L = issued - kStages < 0 ? 0 : issued - kStages; L < issued; ++L)
-        mbar_wait(smem_u32(&bar_full[L % kStages]), (L / kStages) & 1, a.err);
-    }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t fmt = BF16 ? 1u : 0u;
-      const uint32_t idesc1 = (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kDP >> 3) << 17) |
-                              ((uint32_t)(kRows >> 4) << 24);
-      const uint32_t idesc2 = (1u << 4) | ((uint32_t)(m >> 3) << 17) | ((uint32_t)(kRows >> 4) << 24);
-      const uint32_t rot_base = smem_u32(rot);
-      const uint32_t s_base = smem_u32(smat);
-      const uint32_t s_lbo = (uint32_t)(m / 8) * 128u;
-      for (int L = 0;; ++L) {
-        const int64_t tile = blockIdx.x + (int64_t)L * G;
-        const bool have = tile < a.n_tiles;
-        if (have) {
-          // u = (H D) x into slot 256 (L & 1); its previous content, the residual
-          // of tile L - 2, has been consumed once that tile's S r completed
-          const int s = L % kStages, b = L & 1;
-          if (!mbar_wait(smem_u32(&bar_full[s]), (L / kStages) & 1, a.err)) break;
-          if (L >= 2 && !mbar_wait(smem_u32(&bar_zf[b]), ((L - 2) >> 1) & 1, a.err)) break;
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(stages + s * kTileBytes);
-          const uint32_t d_tmem = tmem + (uint32_t)b * 256u;
-#pragma unroll
-          for (int t = 0; t < kDP / 16; ++t) {
-            const uint64_t ad = desc_sw128(a_base + (uint32_t)(t >> 2) * (kTileBytes / 2) + (uint32_t)(t & 3) * 32u);
-            const uint64_t bd = desc_noswz(rot_base + (uint32_t)(2 * t) * 2048u, 2048u, 128u);
-            mma_ss(d_tmem, ad, bd, idesc1, t > 0 ? 1u : 0u);
-          }
-          tc_commit(smem_u32(&bar_empty[s]));
-          tc_commit(smem_u32(&bar_accf[b]));
-        }
-        if (L >= 1) {
-          // z = S r of tile L - 1, once its residual is written and the signs of
-          // tile L - 3 (same z slot) have been read
-          const int Lp = L - 1, b = Lp & 1;
-          if (!mbar_wait(smem_u32(&bar_aready[b]), (Lp >> 1) & 1, a.err)) break;
-          if (Lp >= 2 && !mbar_wait(smem_u32(&bar_zempty[b]), ((Lp - 2) >> 1) & 1, a.err)) break;
-          tc_fence_after();
-          const uint32_t a_tmem = tmem + (uint32_t)b * 256u;
-          const uint32_t z_tmem = a_tmem + 128u;
-#pragma unroll
-          for (int pass = 0; pass < 2; ++pass) {  // hi, then lo parts of r
-#pragma unroll
-            for (int t = 0; t < kDP / 16; ++t) {
-              const uint32_t acol = (uint32_t)(32 * (t >> 1) + 16 * pass + 8 * (t & 1));
-              const uint64_t bd = desc_noswz(s_base + (uint32_t)(2 * t) * s_lbo, s_lbo, 128u);
-              mma_ts(z_tmem, a_tmem + acol, bd, idesc2, (pass | t) ? 1u : 0u);
-            }
-          }
-          tc_commit(smem_u32(&bar_zf[b]));
-        }
-        if (!have) break;
-      }
-      tc_commit(smem_u32(&bar_done));
-      mbar_wait(smem_u32(&bar_done), 0, a.err);
-    }
-  } else {
-    // ---------------------------------------------------------------- epilogue
-    const int ew = warp - 2;        // 0..15
-    const int cg = ew >> 2;         // column group: chunks CPT cg .. CPT cg + CPT - 1
-    const int quarter = warp & 3;   // TMEM lanes 32*quarter .. +31
-    const int rloc = quarter * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const int half_levels = 1 << (K - 1);
-    float tc[4], dc[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) tc[j] = dc[j] = 0.f;
-    const float c0s = 1024.0f * qp.centroids[half_levels];
-#pragma unroll
-    for (int j = 0; j < 3; ++j) {
-      if (j < half_levels - 1) {
-        tc[j] = 1024.0f * qp.boundaries[half_levels + j] - c0s;
-        dc[j] = 1024.0f * (qp.centroids[half_levels + j + 1] - qp.centroids[half_levels + j]);
-      }
-    }
-    const int sw_words = m / 32;  // sign words per vector (2 or 4)
-    // previous tile's row state: its signs and residual norm are written one
-    // tile later
-    int64_t slot_p = 0;
-    bool valid_p = false, zero_p = false;
-
-    // read z of tile Lp and write this thread's sign word
-    auto signs_of = [&](int Lp) -> bool {
-      const int b = Lp & 1;
-      if (!mbar_wait_warp(smem_u32(&bar_zf[b]), (Lp >> 1) & 1, a.err)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < CPT; ++cc) {
-        const int c = CPT * cg + cc;
-        if (c < sw_words) {
-          uint32_t z[32];
-          tmem_ld32_sync(tmem + (uint32_t)b * 256u + 128u + (uint32_t)(32 * c) + lane_off, z);
-          uint32_t neg = 0;
-#pragma unroll
-          for (int i = 31; i >= 0; --i) neg = shift_in(neg, z[i]);
-          // bit i = [(S r)_(32c+i) >= 0]; a zero vector's residual was formed
-          // with the opposite sign (see quant32_prod_sb)
-          const uint32_t word = zero_p ? neg : ~neg;
-          if (valid_p) a.signs[slot_p * sw_words + c] = word;
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&bar_zempty[b]));
-      return true;
-    };
-    // residual norm of the previous tile from the TPR partial squares (the
-    // caller has acquired a barrier that every warp passed after writing them)
-    auto rnorm_of = [&](int Lp) {
-      if (cg == 0 && valid_p) {
-        const float4 q = *reinterpret_cast<const float4*>(&rr_part[Lp & 1][rloc][0]);
-        const float t = TPR == 4 ? (q.x + q.y) + (q.z + q.w) : q.x + q.y;
-        put_rnorm(a.rnorms, slot_p, t > 0.f ? t * rsqrtf(t) * (1.0f / 1024.0f) : 0.f, qp.rnorm_f16);
-      }
-    };
-
-    int L = 0;
-    bool ok = true;
-    for (;; ++L) {
-      const int64_t tile = blockIdx.x + (int64_t)L * G;
-      if (tile >= a.n_tiles) break;
-      const int b = L & 1;
-      if (!mbar_wait_warp(smem_u32(&bar_accf[b]), (L >> 1) & 1, a.err)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t ucol = tmem + (uint32_t)b * 256u + (uint32_t)(32 * CPT * cg) + lane_off;
-      uint32_t ur[CPT][32];
-#pragma unroll
-      for (int cc = 0; cc < CPT; ++cc) tmem_ld32_sync(ucol + (uint32_t)(32 * cc), ur[cc]);
-      {
-        uint64_t s2a = 0, s2b = 0;
-#pragma unroll
-        for (int cc = 0; cc < CPT; ++cc)
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const uint64_t p0 = pk2(__uint_as_float(ur[cc][i]), __uint_as_float(ur[cc][i + 1]));
-            const uint64_t p1 = pk2(__uint_as_float(ur[cc][i + 2]), __uint_as_float(ur[cc][i + 3]));
-            s2a = fma2(p0, p0, s2a);
-            s2b = fma2(p1, p1, s2b);
-          }
-        const float2 fa = upk2(s2a), fb = upk2(s2b);
-        ss_part[b][rloc][cg] = (fa.x + fa.y) + (fb.x + fb.y);
-      }
-      mbar_arrive(smem_u32(&bar_normx));
-      const int64_t row = tile * kRows + rloc;
-      const bool valid = row < a.n_vec;
-      const int64_t seg = valid ? (int64_t)fastdiv((uint32_t)row, a.seg_div) : 0;
-      const int64_t slot = seg * a.seg_cap + (valid ? row - seg * a.seg_len : 0);
-      if (!mbar_wait_warp(smem_u32(&bar_normx), (uint32_t)L & 1u, a.err)) { ok = false; break; }
-      // every warp wrote its partials of tile L - 1 before arriving here
-      if (L >= 1) rnorm_of(L - 1);
-      const float4 q = *reinterpret_cast<const float4*>(&ss_part[b][rloc][0]);
-      const float ss = TPR == 4 ? (q.x + q.y) + (q.z + q.w) : q.x + q.y;  // ||u||^2 = d_pad ||x||^2
-      const bool zero = !(ss > 0.f);
-      const float rs = rsqrtf(ss);
-      const float nu = zero ? 0.f : ss * rs;
-      const float inv = zero ? 0.f : 1024.0f * rs;
-      uint32_t NS[CPT], T0[CPT], T1[CPT], T2[CPT];
-      uint64_t rr2 = 0;
-#pragma unroll
-      for (int cc = 0; cc < CPT; ++cc) {
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(ur[cc][i]);
-        NS[cc] = T0[cc] = T1[cc] = T2[cc] = 0;
-        quant32_prod_sb<K>(v, tc, dc, c0s, inv, NS[cc], T0[cc], T1[cc], T2[cc]);
-        // 2^10 r as fp16 hi (columns 32c .. 32c+15) and lo (32c+16 .. 32c+31)
-        // parts: |r| <= 2, hi keeps the top 11 significant bits (exact in
-        // fp16), lo = 2^10 r - hi is rounded to fp16, about 22 bits in all.
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          uint32_t hiw[8], low[8];
-#pragma unroll
-          for (int qq = 0; qq < 8; ++qq) {
-            const float r0 = v[16 * g + 2 * qq], r1 = v[16 * g + 2 * qq + 1];
-            const float h0 = __uint_as_float(__float_as_uint(r0) & 0xFFFFE000u);
-            const float h1 = __uint_as_float(__float_as_uint(r1) & 0xFFFFE000u);
-            const uint64_t rp = pk2(r0, r1);
-            rr2 = fma2(rp, rp, rr2);
-            const float2 lo = upk2(sub2(rp, pk2(h0, h1)));
-            const __half2 hv = __floats2half2_rn(h0, h1);
-            const __half2 lv = __floats2half2_rn(lo.x, lo.y);
-            hiw[qq] = *reinterpret_cast<const uint32_t*>(&hv);
-            low[qq] = *reinterpret_cast<const uint32_t*>(&lv);
-          }
-          tmem_st8(ucol + (uint32_t)(32 * cc + 8 * g), hiw);
-          tmem_st8(ucol + (uint32_t)(32 * cc + 16 + 8 * g), low);
-        }
-      }
-      const float2 rrf = upk2(rr2);
-      const float rr = rrf.x + rrf.y;
-      rr_part[b][rloc][cg] = rr;
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      tc_fence_before();
-      mbar_arrive(smem_u32(&bar_aready[b]));
-      if (valid) {
-        uint32_t* dst = a.codes + slot * (int64_t)(K * 4) + CPT * cg;
-#pragma unroll
-        for (int cc = 0; cc < CPT; ++cc) {
-          const uint32_t S = zero ? 0u : ~NS[cc];
-          const uint32_t M0 = K == 3 ? (T0[cc] ^ T1[cc] ^ T2[cc]) : T0[cc];
-          uint32_t planes[K];
-          planes_from<K>(S, M0, T1[cc], 0u, planes);
-#pragma unroll
-          for (int p = 0; p < K; ++p) dst[4 * p + cc] = planes[p];
-        }
-        if (cg == 0) a.norms[slot] = nu * qp.inv_sqrt_dpad;
-      }
-      // signs of the previous tile: its S r ran while this tile was quantized
-      if (L >= 1 && !signs_of(L - 1)) { ok = false; break; }
-      slot_p = slot;
-      valid_p = valid;
-      zero_p = zero;
-    }
-    if (ok && L >= 1) {
-      // the last tile: its partial squares were written before aready
-      if (mbar_wait_warp(smem_u32(&bar_aready[(L - 1) & 1]), ((L - 1) >> 1) & 1, a.err)) {
-        rnorm_of(L - 1);
-        signs_of(L - 1);
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols));
-  }
-}
 
 // ------------------------------------------------------------------ Q_prod, one thread per vector
 

@@ -427,10 +427,10 @@ tq_status tq_params_tables(const tq_params* p, float* centroids, float* boundari
 
 // ------------------------------------------------------------------ attention feature coefficients
 
-#include "tq_attn2.h"
+#include "tq_attn_params.h"
 
 namespace tq {
-namespace attn2 {
+namespace attn {
 
 void odd_feature_coefs(const float* centroids, int k, float* alpha, float* alpha_sum) {
   // subsets as bit masks in the kernel's order
@@ -477,5 +477,5 @@ void odd_feature_coefs(const float* centroids, int k, float* alpha, float* alpha
   *alpha_sum = (float)s;
 }
 
-}  // namespace attn2
+}  // namespace attn
 }  // namespace tq

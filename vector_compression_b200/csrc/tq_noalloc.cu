@@ -5,8 +5,6 @@
 // allocating library routine.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "tq_internal.h"
 
 namespace {
@@ -14,24 +12,17 @@ namespace {
 // One array per device that loads the library, held until the process exits.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[TQ_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 128;
-void* g_scratch_ptr[kMaxDevices];  // device address of the array, per device
-std::mutex g_scratch_mu;
-
-// Host code only sees a stand-in for the array's name, not a device address:
-// look the address up once per device, with that device current.
+// Host code only sees a stand-in for the array's name, not a device address.
+// The address is looked up on every call, with the caller's device and
+// context current, so it is always the array of the context the kernels
+// will run in: a cached address would go stale after cudaDeviceReset or
+// belong to another context when the caller switches contexts.  The lookup
+// allocates nothing; the first lookup in a context may load the library's
+// module into it, so that first call should come before any stream capture.
 tq_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return TQ_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return TQ_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return TQ_ERR_CUDA;
+  *out = p;
   return TQ_OK;
 }
 
