@@ -436,6 +436,7 @@ def main():
                        "key_bits": cfg.key_bits, "value_bits": cfg.value_bits, "qjl_m": kp.m, "value_scale": args.value_scale,
                        "rnorm_dtype": kp.rnorm_dtype,
                        "rotation": "randomized Hadamard", "l2": "inputs larger than L2 (no flush)",
+                       "arithmetic": ARITHMETIC,
                        "bytes_per_step": step_bytes, "parallelism": f"replica x{world}"},
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["GB/s"], "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": kernels[dom]["frac_of_hbm"],
@@ -452,6 +453,17 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+# What the path computes in, beside the line's "dtype" (the type of the
+# stored norms, scores and outputs).
+ARITHMETIC = {
+    "encode": "fp32; rotation and S r as tcgen05 MMAs (exact +-1 fp16 rotation entries, fp16 S, "
+              "residual split fp16 hi + lo), fp32 accumulation",
+    "attention": "exact integer tensor-core contractions of code bits against fixed-point operands: "
+                 "queries q' and S q' 24-bit per head, softmax weights p ||v|| 16-bit per head and "
+                 "384-token sub-chunk; fp32 softmax, norms and folds",
+}
 
 
 def source_hash():
