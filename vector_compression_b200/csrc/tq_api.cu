@@ -17,6 +17,7 @@
 #include "tq_enc3.h"
 #include "tq_gemm.cuh"
 #include "tq_internal.h"
+#include "tq_score_tc.h"
 #include "tq_scores.cuh"
 #include "tq_wait.cuh"
 
@@ -567,7 +568,10 @@ tq_status tq_scores_workspace_size(const tq_params* kp, int64_t nq, int64_t n_ve
                                    size_t* bytes) {
   if (!kp || !bytes || nq < 0 || n_vec < 0 || topk < 0) return TQ_ERR_INVALID_ARG;
   size_t b = tq::round_up((size_t)nq * kp->q.d_pad * 4, 256) + tq::round_up((size_t)nq * kp->q.m * 4, 256);
-  if (topk > 0) b += tq::round_up((size_t)nq * n_vec * 4, 256);
+  if (tq::score_tc::covers(kp->q, topk))
+    b += tq::score_tc::workspace_bytes(kp->q, nq, n_vec, topk);  // no score matrix: the top-k is fused
+  else if (topk > 0)
+    b += tq::round_up((size_t)nq * n_vec * 4, 256);
   *bytes = b;
   return TQ_OK;
 }
@@ -590,9 +594,15 @@ tq_status tq_scores(const tq_params* kp, const float* q, int64_t nq, int64_t ldq
   w += tq::round_up((size_t)nq * kp->q.d_pad * 4, 256);
   float* u = (float*)w;
   w += tq::round_up((size_t)nq * kp->q.m * 4, 256);
-  float* full = topk > 0 ? (float*)w : scores;
   int e = tq::launch_query_prep(kp->q, q, nq, ldq, qrot, u, stream);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
+  // the tensor-core scorer (fused top-k) whenever it covers the shape
+  if (tq::score_tc::covers(kp->q, topk) && tq::aligned16(signs)) {
+    e = tq::score_tc::launch(kp->q, qrot, u, nq, codes, signs, norms, rnorms, n_vec, scores, topk, top_s, top_i, w,
+                             tq::device_error_ptr(), tq::num_sms(), tq::S(stream));
+    return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  }
+  float* full = topk > 0 ? (float*)w : scores;
   e = tq::launch_scores(kp->q, qrot, u, nq, codes, signs, norms, rnorms, n_vec, full, stream);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
   if (topk > 0) {
