@@ -132,3 +132,51 @@ def test_retrieval_full_size(bits):
         order = np.lexsort((np.arange(n), -s[r]))[:R["topk"]]
         assert np.array_equal(top_i[r].cpu().numpy(), order)
         assert np.array_equal(top_s[r].cpu().numpy(), s[r, order])
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_retrieval_1024_queries_fused_topk_and_recall(bits):
+    # The retrieval workload at its stated size: 1e6 x 1536 unit vectors,
+    # 1024 unit queries, top-10 of the unbiased estimator with the fused
+    # top-k (no score matrix), and recall@10 against the exact fp32 products.
+    R = synth.RETRIEVAL
+    d, n = R["d"], R["n"]
+    ora, lib = make_pair(d, bits, True, seed=R["seed"], m=R["m"], dense=True)
+    x = synth.gaussian_vectors(n, d, seed=R["seed"], device=DEV, n_outliers=R["n_outliers"],
+                               outlier_scale=R["outlier_scale"], normalize=True)
+    qs = synth.gaussian_vectors(R["n_queries"], d, seed=R["seed"] + 1, device=DEV, normalize=True)
+    codes, signs, norms, rnorms = tq.tq_encode_prod(lib, x)
+    _, top_s, top_i = tq.tq_scores(lib, qs, codes, signs, norms, rnorms, topk=R["topk"], want_scores=False)
+    # the first 64 queries again with their score rows
+    sc, ts64, ti64 = tq.tq_scores(lib, qs[:64], codes, signs, norms, rnorms, topk=R["topk"])
+    torch.cuda.synchronize()
+    tq.tq_sync_check()
+    assert np.array_equal(top_i[:64].cpu().numpy(), ti64.cpu().numpy())
+    assert np.array_equal(top_s[:64].cpu().numpy(), ts64.cpu().numpy())
+    s = sc.cpu().numpy()
+    for r in range(0, 64, 9):
+        order = np.lexsort((np.arange(n), -s[r]))[:R["topk"]]
+        assert np.array_equal(ti64[r].cpu().numpy(), order)
+    # sampled scores against the oracle (1e-3 of max(|s|, n |q| / sqrt(d)))
+    rng = np.random.default_rng(13)
+    idx = np.sort(rng.choice(n, size=256, replace=False))
+    e = ora.encode(x_np(x[torch.from_numpy(idx).to(DEV)]))
+    gi = o.unpack_row(u32(codes[idx]), ora.k, ora.d_pad)
+    _, bad = check_codes(gi, e["idx"], e["y"], ora.boundaries, d)
+    sig_bad = (o.unpack_signs(u32(signs[idx]), ora.m) != o.unpack_signs(e["signs"], ora.m)).any(axis=1)
+    qn = x_np(qs[:64])
+    want = ora.scores(qn, e["idx"], e["norms"], e["signs"], e["rnorms"])
+    floor = e["norms"][None, :] * np.linalg.norm(qn, axis=1)[:, None] / math.sqrt(d)
+    ok = ~(bad | sig_bad)
+    assert_close_rel(s[:, idx][:, ok], want[:, ok], floor[:, ok], what="scores")
+    # recall@10 of the estimator's top-10 against the exact fp32 top-10
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    hits = 0
+    for a in range(0, qs.shape[0], 128):
+        exact = torch.topk(qs[a:a + 128] @ x.T, R["topk"], dim=1).indices
+        hits += int((exact.unsqueeze(2) == top_i[a:a + 128].unsqueeze(1)).any(dim=2).sum().item())
+    torch.backends.cuda.matmul.allow_tf32 = prev
+    recall = hits / (qs.shape[0] * R["topk"])
+    print(f"retrieval b={bits}: recall@10 = {recall:.3f} over {qs.shape[0]} queries")
+    assert recall > 0.05  # a random top-10 of 1e6 would score ~1e-5
