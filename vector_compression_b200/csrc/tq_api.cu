@@ -597,7 +597,8 @@ tq_status tq_scores(const tq_params* kp, const float* q, int64_t nq, int64_t ldq
   int e = tq::launch_query_prep(kp->q, q, nq, ldq, qrot, u, stream);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
   // the tensor-core scorer (fused top-k) whenever it covers the shape
-  if (tq::score_tc::covers(kp->q, topk) && tq::aligned16(signs)) {
+  if (tq::score_tc::covers(kp->q, topk)) {
+    if (!tq::aligned16(signs) || !tq::aligned16(codes)) return TQ_ERR_INVALID_ARG;
     e = tq::score_tc::launch(kp->q, qrot, u, nq, codes, signs, norms, rnorms, n_vec, scores, topk, top_s, top_i, w,
                              tq::device_error_ptr(), tq::num_sms(), tq::S(stream));
     return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;

@@ -63,9 +63,14 @@ constexpr float kFix = 8323072.0f;           // 2^23 - 2^16: three balanced sign
 // D[tile] = [MSE part 96 | sign part 96]
 constexpr uint32_t kTA = 0, kTD = 128, kTDT = 2 * kNP;
 
-// shared memory: B ring | candidate scores [kQB][kGroup] | top lists | headers
+// per-thread ring of code words in flight (cp.async): kPD chunks ahead
+constexpr int kPD = 8;
+
+// shared memory: B ring | code ring [kPD][kGroup][4 words] | candidate
+// scores [kQB][kGroup] | top lists | headers
 constexpr uint32_t kOffB = 0;
-constexpr uint32_t kOffCand = kOffB + kBStages * kChunkBytes;
+constexpr uint32_t kOffRing = kOffB + kBStages * kChunkBytes;
+constexpr uint32_t kOffCand = kOffRing + kPD * kGroup * 16;
 constexpr uint32_t kOffTopS = kOffCand + kQB * kGroup * 4;
 constexpr uint32_t kOffTopI = kOffTopS + kQB * kMaxTopk * 4;
 constexpr uint32_t kOffHdr = kOffTopI + kQB * kMaxTopk * 8;
@@ -160,6 +165,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t* r) {
       : "r"(addr)
       : "memory");
 }
+
+// asynchronous global -> shared copies of 4 or 16 bytes (per thread)
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // (score, index) order of the top-k: score descending, then index ascending
 __device__ __forceinline__ bool better(float s1, int64_t i1, float s2, int64_t i2) {
@@ -410,24 +429,39 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(Args a) {
       ++ws;
       return r_ok;
     };
-    // the 4 A words of chunk c for vector v (zero when v is past the range)
-    auto chunk_words = [&](int64_t v, bool valid, int c, uint32_t (&w)[4]) {
-      if (!valid) {
-        w[0] = w[1] = w[2] = w[3] = 0u;
-        return;
-      }
+    // The raw words of chunk c of vector v go to ring slot c % kPD: the sign
+    // words, or the plane words that make its four feature words (fk = 1: 4
+    // plane words; fk = 2: planes 0, 1 of 2 plane-word positions; fk = 4:
+    // planes 0..2 of one position).
+    const uint32_t ring = s_base + kOffRing + (uint32_t)t_id * 16;
+    auto issue_chunk = [&](int64_t v, int c) {
+      const uint32_t dst = ring + (uint32_t)(c % kPD) * (kGroup * 16);
       if (c >= a.n_mse) {
-        const uint4 x = *reinterpret_cast<const uint4*>(a.signs + v * a.sw + 4 * (c - a.n_mse));
-        w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+        cp_async16(dst, a.signs + v * a.sw + 4 * (c - a.n_mse));
         return;
       }
-      const uint32_t* row_w = a.codes + v * KW;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int wd = 4 * c + i, cw = wd / a.fk, f = wd % a.fk;
-        uint32_t pl[3] = {0u, 0u, 0u};
-        for (int p = 0; p < a.kk; ++p) pl[p] = __ldg(row_w + p * a.wpp + cw);
-        w[i] = feature_word(pl, a.kk, f);
+      const uint32_t* rw = a.codes + v * KW;
+      if (a.fk == 1) {
+        cp_async16(dst, rw + 4 * c);
+      } else if (a.fk == 2) {
+        cp_async8(dst, rw + 2 * c);
+        cp_async8(dst + 8, rw + a.wpp + 2 * c);
+      } else {
+        cp_async4(dst, rw + c);
+        cp_async4(dst + 4, rw + a.wpp + c);
+        cp_async4(dst + 8, rw + 2 * a.wpp + c);
+      }
+    };
+    // the four A words of chunk c (in order: feature f of position cw at
+    // 4 c + i = cw fk + f) from its ring slot
+    auto read_chunk = [&](int c, uint32_t (&w)[4]) {
+      const uint4 r = *reinterpret_cast<const uint4*>(smem + kOffRing + (c % kPD) * (kGroup * 16) + t_id * 16);
+      if (c >= a.n_mse || a.fk == 1) {
+        w[0] = r.x; w[1] = r.y; w[2] = r.z; w[3] = r.w;
+      } else if (a.fk == 2) {  // r = plane 0 of (cw0, cw1), plane 1 of (cw0, cw1)
+        w[0] = r.x; w[1] = r.z; w[2] = r.y; w[3] = r.w;
+      } else {                 // r = planes 0, 1, 2 of one position
+        w[0] = r.x; w[1] = r.y; w[2] = r.z; w[3] = r.x ^ r.y ^ r.z;
       }
     };
     for (int64_t item = i0; ok && item < i1; ++item, ++it) {
@@ -446,10 +480,19 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(Args a) {
       for (int64_t g = 0; ok && g < groups; ++g, ++gc) {
         const int64_t v = v0 + g * kGroup + t_id;
         const bool valid = v < v1;
-        uint32_t wcur[4];
-        chunk_words(v, valid, 0, wcur);
+        // kPD chunks in flight (one copy group per chunk, empty past the end)
+        for (int c = 0; c < kPD; ++c) {
+          if (valid && c < nc) issue_chunk(v, c);
+          cp_commit();
+        }
         for (int c = 0; c < nc; ++c, ++cc) {
           const uint32_t buf = cc & 1;
+          uint32_t wcur[4] = {0u, 0u, 0u, 0u};
+          cp_wait<kPD - 1>();  // chunk c's copies have landed
+          if (valid) read_chunk(c, wcur);
+          __syncwarp();        // the slot's reads are done before it is refilled
+          if (valid && c + kPD < nc) issue_chunk(v, c + kPD);
+          cp_commit();
           if (cc >= 2 && !wait_bar_warp(B(bar_afree[buf]), ((cc - 2) >> 1) & 1, a.err)) { ok = false; break; }
           uint32_t reg[32];
 #pragma unroll
@@ -457,12 +500,12 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(Args a) {
 #pragma unroll
             for (int s = 0; s < 8; ++s) reg[8 * i + s] = (wcur[i] >> s) & 0x01010101u;
           tmem_st32(tmem + kTA + (buf * 2 + tile) * 32 + lane_off, reg);
-          if (c + 1 < nc) chunk_words(v, valid, c + 1, wcur);
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(B(bar_afull[buf]));
         }
+        cp_wait<0>();  // nothing of this group stays in flight (error exit)
         if (!ok) break;
         // ---- the group's scores
         if (!wait_bar_warp(B(bar_dfull), gc & 1, a.err)) { ok = false; break; }
