@@ -1,7 +1,8 @@
 """Scores and fused top-k on the tensor cores versus the oracle: many query
 blocks (a partial last block), ragged vector counts (a partial last group of
 two 128-vector tiles), Hadamard and dense rotations, key codes of 1..3 bits,
-top-k of 1..32 with and without the full score matrix.  The caches hold the
+top-k of 1..32 with and without the full score matrix, and more work items
+than SMs.  The caches hold the
 oracle's codes, so scores are compared element by element at 1e-5 relative;
 the top-k must be the exact (score descending, index ascending) top-k of the
 GPU's own scores."""
@@ -32,6 +33,10 @@ def _dev(a):
     (128, False, 4, 777, 64, 32),     # the largest top-k
     (256, True, 4, 700, 40, 10),      # dense rotation, m = 256, k = 3 (four features)
     (256, True, 2, 513, 31, 5),       # dense, k = 1, one partial query block
+    # 33 query blocks x 12 ranges of 2 groups: more items than SMs, so a CTA
+    # runs consecutive items of one query block (its lists carry over) and
+    # crosses into the next block
+    (128, False, 3, 6000, 1050, 10),
 ])
 def test_tc_scores_and_topk(d, dense, bits, n, nq, topk):
     ora, lib = make_pair(d, bits, True, seed=70 + bits, dense=dense)

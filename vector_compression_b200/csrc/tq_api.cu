@@ -292,9 +292,17 @@ int launch_query_prep(const QParams& qp, const float* q, int64_t nq, int64_t ldq
   const unsigned blocks = (unsigned)ceil_div(nq, 4);
   if (nq == 0) return cudaSuccess;
   if (qp.rot == TQ_ROT_DENSE) {
-    query_prep_dense_kernel<<<blocks, 128, 4 * 2 * qp.d * sizeof(float), st>>>(qp, q, nq, ldq,
-                                                                               qrot, u);
-    return cudaGetLastError();
+    // q' = Pi q and u = S q' as tiled GEMMs over all queries (rows of up to
+    // 2^20 queries per launch keep the grid inside its limits)
+    if (ldq > INT32_MAX) return cudaErrorInvalidValue;
+    for (int64_t r0 = 0; r0 < nq; r0 += (int64_t)1 << 20) {
+      const int rows = (int)std::min<int64_t>(nq - r0, (int64_t)1 << 20);
+      float* qr = qrot + r0 * qp.d;
+      cudaError_t e = gemm_abt_f32(q + r0 * ldq, qp.Pi, qr, rows, qp.d, qp.d, st, (int)ldq);
+      if (e == cudaSuccess && u) e = gemm_abt_f32(qr, qp.S, u + r0 * qp.m, rows, qp.m, qp.d, st);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
   }
   switch (qp.d_pad / 32) {
 #define TQ_QP(AA)                                                                                \

@@ -1,6 +1,7 @@
-// fp32 GEMM C[M][N] = A[M][K] * B[N][K]^T (all row-major), used by the
-// dense-rotation path: y = x Pi^T (Pi row-major, y = Pi x per vector) and
-// z = r S^T.  SIMT with 128x128 CTA tiles, 8x8 outputs per thread, K tiles of
+// fp32 GEMM C[M][N] = A[M][K] * B[N][K]^T (row-major; A rows lda apart), used
+// by the dense-rotation path: y = x Pi^T (Pi row-major, y = Pi x per vector),
+// z = r S^T, and the query side q' = Pi q, u = S q'.  Each output sums its K
+// products in ascending k order.  SIMT with 128x128 CTA tiles, 8x8 outputs per thread, K tiles of
 // 16 staged through shared memory.  M, N, K arbitrary (bounds-checked).
 #pragma once
 
@@ -10,10 +11,11 @@ namespace tq {
 
 constexpr int kGemmBM = 128, kGemmBN = 128, kGemmBK = 16;
 
+template <bool kStridedA>
 __global__ void __launch_bounds__(256) gemm_abt_f32_kernel(const float* __restrict__ A,
                                                            const float* __restrict__ B,
                                                            float* __restrict__ C, int M, int N,
-                                                           int K) {
+                                                           int K, int lda) {
   __shared__ float As[kGemmBK][kGemmBM + 4];
   __shared__ float Bs[kGemmBK][kGemmBN + 4];
   const int tid = threadIdx.x;
@@ -31,7 +33,7 @@ __global__ void __launch_bounds__(256) gemm_abt_f32_kernel(const float* __restri
       const int e = tid + 256 * r;
       const int row = e / kGemmBK, kk = e % kGemmBK;
       const int gm = m0 + row, gn = n0 + row, gk = k0 + kk;
-      As[kk][row] = (gm < M && gk < K) ? A[(size_t)gm * K + gk] : 0.f;
+      As[kk][row] = (gm < M && gk < K) ? A[(size_t)gm * (kStridedA ? lda : K) + gk] : 0.f;
       Bs[kk][row] = (gn < N && gk < K) ? B[(size_t)gn * K + gk] : 0.f;
     }
     __syncthreads();
@@ -62,10 +64,13 @@ __global__ void __launch_bounds__(256) gemm_abt_f32_kernel(const float* __restri
 }
 
 inline cudaError_t gemm_abt_f32(const float* A, const float* B, float* C, int M, int N, int K,
-                                cudaStream_t st) {
+                                cudaStream_t st, int lda = -1) {
   if (M <= 0 || N <= 0) return cudaSuccess;
   dim3 grid((N + kGemmBN - 1) / kGemmBN, (M + kGemmBM - 1) / kGemmBM);
-  gemm_abt_f32_kernel<<<grid, 256, 0, st>>>(A, B, C, M, N, K);
+  if (lda < 0 || lda == K)
+    gemm_abt_f32_kernel<false><<<grid, 256, 0, st>>>(A, B, C, M, N, K, K);
+  else
+    gemm_abt_f32_kernel<true><<<grid, 256, 0, st>>>(A, B, C, M, N, K, lda);
   return cudaGetLastError();
 }
 

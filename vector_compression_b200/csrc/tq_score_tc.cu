@@ -19,21 +19,21 @@
 // three columns.
 // Products and sums are exact integers.
 //
-// The query operands are built once per call (query_image_kernel), per block
-// of 32 queries: a header with the per-query constants and B in chunks of
-// 128 K bytes x 96 rows.  The scoring kernel is persistent: a work item is
-// one query block and a range of vectors, in groups of two 128-vector tiles
-// that share every B chunk.  Warp 0 stages the B chunks with bulk copies
-// (the images stay in L2), warps 1 and 10 issue the MMAs of tile 0 and tile
-// 1 (one thread issues one MMA per ~60 cycles, so the two tiles get one
-// issuer each), warps 2..9 are the workers: each thread owns one vector (one
-// TMEM lane), loads its code words, writes the expanded bits to tensor memory
-// with tcgen05.st, and after the group's last chunk folds its row of D into
-// 32 scores.  With a top-k requested the scores never leave the SM: each
-// query keeps its best k (score descending, index ascending) in shared
-// memory, merged per group by one warp per query; the item's lists go to the
-// workspace and a final kernel merges the items of each query.  Every wait
-// is bounded (error word + clean exit).
+// The query operands are built once per call (query_scale_kernel, then
+// query_digits_kernel), per block of 32 queries: a header with the per-query
+// constants and B in chunks of 128 K bytes x 96 rows.  The scoring kernel is
+// persistent: a work item is one query block and a range of vectors, in groups
+// of two 128-vector tiles that share every B chunk.  Warp 0 stages the B
+// chunks with bulk copies (the images stay in L2), warps 1 and 10 issue the
+// MMAs of tile 0 and tile 1 (one thread issues one MMA per ~60 cycles, so the
+// two tiles get one issuer each), warps 2..9 are the workers: each thread owns
+// one vector (one TMEM lane), loads its code words, writes the expanded bits
+// to tensor memory with tcgen05.st, and after the group's last chunk folds its
+// row of D into 32 scores.  With a top-k requested the scores never leave the
+// SM: each query keeps its best k (score descending, index ascending) in
+// shared memory, merged per group by one warp per query; the item's lists go
+// to the workspace and a final kernel merges the items of each query.  Every
+// wait is bounded (error word + clean exit).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -67,13 +67,16 @@ constexpr uint32_t kTA = 0, kTD = 128, kTDT = 2 * kNP;
 constexpr int kPD = 8;
 
 // shared memory: B ring | code ring [kPD][kGroup][4 words] | candidate
-// scores [kQB][kGroup] | top lists | headers
+// scores [kQB][kGroup] | top lists | survivor masks | thresholds | headers
 constexpr uint32_t kOffB = 0;
 constexpr uint32_t kOffRing = kOffB + kBStages * kChunkBytes;
 constexpr uint32_t kOffCand = kOffRing + kPD * kGroup * 16;
 constexpr uint32_t kOffTopS = kOffCand + kQB * kGroup * 4;
 constexpr uint32_t kOffTopI = kOffTopS + kQB * kMaxTopk * 4;
-constexpr uint32_t kOffHdr = kOffTopI + kQB * kMaxTopk * 8;
+constexpr uint32_t kOffMask = kOffTopI + kQB * kMaxTopk * 8;  // [kQB][8] survivor bits per warp
+constexpr uint32_t kOffThrS = kOffMask + kQB * 8 * 4;          // [kQB] k-th best score
+constexpr uint32_t kOffThrI = kOffThrS + kQB * 4;              // [kQB] its index
+constexpr uint32_t kOffHdr = kOffThrI + kQB * 8;
 constexpr uint32_t kSmem = kOffHdr + 2 * kHdr;
 
 struct Args {
@@ -112,8 +115,10 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
 }
+// try_wait parks the polling warp in hardware between tests, which leaves
+// the issue slots to the warps doing the work
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, unsigned* err) {
-  return bounded_wait<false>(bar, parity, err);
+  return bounded_wait<true>(bar, parity, err);
 }
 __device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, unsigned* err) {
   return __all_sync(0xffffffffu, wait_bar(bar, parity, err)) != 0;
@@ -211,76 +216,105 @@ __device__ __forceinline__ uint32_t feature_word(const uint32_t* p, int k, int f
 // (word >> s) & 0x01010101).  Sign part: A word w' is sign word w'.  Row n of
 // B = 3 (query) + (digit byte); chunk c of a part holds its K bytes
 // [128 c, 128 c + 128) as 8 x 12 core matrices of 8 rows x 16 bytes.
-__global__ void __launch_bounds__(256) query_image_kernel(QParams kp, Args a, float kalpha0, float kalpha1,
+// Per query and part (one warp each): the fixed-point scale inv = kFix /
+// max|x| over the part's operand values x (alpha_f q'_j for the MSE part, u_i
+// for the signs), stored in qinv, and the header constants of the image,
+// which need the integer sum C of the part's rounded values X = rint(x inv):
+// x = 2 b - 1 on the code side turns sum_j X_j (2 b_j - 1) into 2 D - C.
+__global__ void __launch_bounds__(256) query_scale_kernel(QParams kp, Args a, float kalpha0, float kalpha1,
                                                           float kalpha2, float kalpha3, const float* __restrict__ qrot,
-                                                          const float* __restrict__ u, unsigned char* __restrict__ img) {
-  const int qb = blockIdx.x, tid = threadIdx.x;
+                                                          const float* __restrict__ u, float* __restrict__ qinv,
+                                                          unsigned char* __restrict__ img, int64_t n_qb) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wg = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);  // (query slot, part)
+  if (wg >= n_qb * kQB * 2) return;
+  const int part = (int)(wg & 1);
+  const int64_t qs = wg >> 1, qb = qs / kQB;
+  const int ql = (int)(qs % kQB);
   const int dp = kp.d_pad, m = kp.m;
-  unsigned char* base = img + (size_t)qb * a.img_bytes;
-  __shared__ float s_inv[kQB][2];
-  __shared__ unsigned long long s_C[kQB][2];
   const float alpha[4] = {kalpha0, kalpha1, kalpha2, kalpha3};
   float amax = 0.f;
   for (int f = 0; f < a.fk; ++f) amax = fmaxf(amax, fabsf(alpha[f]));
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int qp = warp; qp < 2 * kQB; qp += 8) {
-    const int ql = qp >> 1, part = qp & 1;
-    const int64_t q = (int64_t)qb * kQB + ql;
-    float mx = 0.f;
-    if (q < a.nq) {
-      if (part == 0)
-        for (int j = lane; j < dp; j += 32) mx = fmaxf(mx, fabsf(qrot[q * dp + j]));
-      else
-        for (int j = lane; j < m; j += 32) mx = fmaxf(mx, fabsf(u[q * m + j]));
-    }
-    mx = warp_max(mx);
-    if (part == 0) mx *= amax;
-    if (lane == 0) {
-      s_inv[ql][part] = mx > 0.f ? kFix / mx : 0.f;
-      s_C[ql][part] = 0ull;
+  const bool live = qs < a.nq;
+  float mx = 0.f;
+  if (live) {
+    if (part == 0)
+      for (int j = lane; j < dp; j += 32) mx = fmaxf(mx, fabsf(qrot[qs * dp + j]));
+    else
+      for (int j = lane; j < m; j += 32) mx = fmaxf(mx, fabsf(u[qs * m + j]));
+  }
+  mx = warp_max(mx);
+  if (part == 0) mx *= amax;
+  const float inv = mx > 0.f ? kFix / mx : 0.f;
+  long long C = 0;
+  if (live && inv > 0.f) {
+    if (part == 0) {
+      for (int f = 0; f < a.fk; ++f)
+        for (int j = lane; j < dp; j += 32) C += __float2int_rn(alpha[f] * qrot[qs * dp + j] * inv);
+    } else {
+      for (int j = lane; j < m; j += 32) C += __float2int_rn(u[qs * m + j] * inv);
     }
   }
-  __syncthreads();
-  const int mse_words = a.fk * a.wpp, kt = (mse_words + a.sw) * 32;
-  for (int64_t e = tid; e < (int64_t)kQB * kt; e += 256) {
-    const int ql = (int)(e / kt), k = (int)(e % kt);
-    const int w = k >> 5, s = (k >> 2) & 7, i = k & 3, cc = 8 * i + s;
-    const int64_t q = (int64_t)qb * kQB + ql;
-    const bool sign = w >= mse_words;
-    int X = 0;
-    if (q < a.nq) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) C += __shfl_xor_sync(0xffffffffu, C, o);
+  if (lane == 0) {
+    qinv[qs * 2 + part] = inv;
+    float* hdr = reinterpret_cast<float*>(img + qb * (int64_t)a.img_bytes) + 4 * ql + 2 * part;
+    const float scale = part == 0 ? 1.0f : kp.kappa;
+    hdr[0] = inv > 0.f ? scale * 2.0f / inv : 0.f;
+    hdr[1] = inv > 0.f ? (float)(-(double)scale * (double)C / (double)inv) : 0.f;
+  }
+}
+
+// The B operand of each query block, in chunks of 128 K bytes x 96 rows (row
+// n = 3 ql + p holds digit p of query ql's values; K-major core matrices of 8
+// rows x 16 bytes).  K byte k of a part's 32-bit word w stands for bit
+// 8 (k & 3) + ((k >> 2) & 7) of that word, the order in which the scorer
+// expands the code words.  One thread per query and 4 consecutive K bytes.
+__global__ void __launch_bounds__(256) query_digits_kernel(QParams kp, Args a, float kalpha0, float kalpha1,
+                                                           float kalpha2, float kalpha3,
+                                                           const float* __restrict__ qrot,
+                                                           const float* __restrict__ u,
+                                                           const float* __restrict__ qinv,
+                                                           unsigned char* __restrict__ img) {
+  const int mse_words = a.fk * a.wpp, kt4 = (mse_words + a.sw) * 8;  // K bytes / 4 per query
+  const int64_t qb = blockIdx.y;
+  const int e = blockIdx.x * 256 + threadIdx.x;
+  if (e >= kQB * kt4) return;
+  const int ql = e / kt4, k = 4 * (e % kt4);
+  const int64_t q = qb * kQB + ql;
+  const int w = k >> 5, s = (k >> 2) & 7;
+  const bool sign = w >= mse_words;
+  const float alpha[4] = {kalpha0, kalpha1, kalpha2, kalpha3};
+  uint32_t dw[3] = {0u, 0u, 0u};
+  if (q < a.nq) {
+    const float inv = qinv[q * 2 + (sign ? 1 : 0)];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int cc = 8 * i + s;
       float x;
       if (!sign) {
         const int f = w % a.fk, cw = w / a.fk;
-        x = alpha[f] * qrot[q * dp + 32 * cw + cc] * s_inv[ql][0];
+        x = alpha[f] * qrot[q * kp.d_pad + 32 * cw + cc] * inv;
       } else {
-        x = u[q * m + 32 * (w - mse_words) + cc] * s_inv[ql][1];
+        x = u[q * kp.m + 32 * (w - mse_words) + cc] * inv;
       }
-      X = __float2int_rn(x);  // |X| <= 2^23 - 2^16
-    }
-    if (X != 0) atomicAdd(&s_C[ql][sign ? 1 : 0], (unsigned long long)(long long)X);
-    const int d0 = ((X + 128) & 0xFF) - 128, x1 = (X - d0) >> 8;
-    const int d1 = ((x1 + 128) & 0xFF) - 128, d2 = (x1 - d1) >> 8;
-    const int kp_ = sign ? k - mse_words * 32 : k;  // K byte within the part
-    unsigned char* chunk = base + kHdr + (uint32_t)((sign ? a.n_mse : 0) + (kp_ >> 7)) * kChunkBytes;
-    const int kk = kp_ & 127;
-#pragma unroll
-    for (int p = 0; p < 3; ++p) {
-      const int n = 3 * ql + p;
-      const int dg = p == 0 ? d0 : p == 1 ? d1 : d2;
-      chunk[((kk >> 4) * (kNP / 8) + (n >> 3)) * 128 + (n & 7) * 16 + (kk & 15)] = (unsigned char)(dg & 0xFF);
+      const int X = __float2int_rn(x);  // |X| <= 2^23 - 2^16: three balanced signed bytes
+      const int d0 = ((X + 128) & 0xFF) - 128, x1 = (X - d0) >> 8;
+      const int d1 = ((x1 + 128) & 0xFF) - 128, d2 = (x1 - d1) >> 8;
+      dw[0] |= (uint32_t)(d0 & 0xFF) << (8 * i);
+      dw[1] |= (uint32_t)(d1 & 0xFF) << (8 * i);
+      dw[2] |= (uint32_t)(d2 & 0xFF) << (8 * i);
     }
   }
-  __syncthreads();
-  if (tid < kQB) {
-    const float qi = s_inv[tid][0], ui = s_inv[tid][1];
-    const double Cq = (double)(long long)s_C[tid][0], Cu = (double)(long long)s_C[tid][1];
-    float4 c;
-    c.x = qi > 0.f ? 2.0f / qi : 0.f;
-    c.y = qi > 0.f ? (float)(-Cq / (double)qi) : 0.f;
-    c.z = ui > 0.f ? kp.kappa * 2.0f / ui : 0.f;
-    c.w = ui > 0.f ? (float)(-(double)kp.kappa * Cu / (double)ui) : 0.f;
-    reinterpret_cast<float4*>(base)[tid] = c;
+  const int kp_ = sign ? k - mse_words * 32 : k;  // K byte within the part
+  unsigned char* chunk =
+      img + qb * (int64_t)a.img_bytes + kHdr + (uint32_t)((sign ? a.n_mse : 0) + (kp_ >> 7)) * kChunkBytes;
+  const int kk = kp_ & 127;
+#pragma unroll
+  for (int p = 0; p < 3; ++p) {
+    const int n = 3 * ql + p;
+    *reinterpret_cast<uint32_t*>(chunk + ((kk >> 4) * (kNP / 8) + (n >> 3)) * 128 + (n & 7) * 16 + (kk & 15)) = dw[p];
   }
 }
 
@@ -418,7 +452,11 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(Args a) {
     float* cand = reinterpret_cast<float*>(smem + kOffCand);       // [kQB][kGroup]
     float* top_s = reinterpret_cast<float*>(smem + kOffTopS);      // [kQB][kMaxTopk]
     int64_t* top_i = reinterpret_cast<int64_t*>(smem + kOffTopI);  // [kQB][kMaxTopk]
+    uint32_t* smask = reinterpret_cast<uint32_t*>(smem + kOffMask);   // [kQB][8]
+    float* thr_s = reinterpret_cast<float*>(smem + kOffThrS);         // [kQB]
+    int64_t* thr_i = reinterpret_cast<int64_t*>(smem + kOffThrI);     // [kQB]
     const int K = a.topk;
+    int64_t prev_qb = -1;
     uint32_t cc = 0, gc = 0, ws = 0;
     int it = 0;
     bool ok = true;
@@ -472,11 +510,21 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(Args a) {
       const int ib = it & 1;
       if (!wait_bar_warp(B(bar_hfull[ib]), (it >> 1) & 1, a.err)) { ok = false; break; }
       const float4* hdr = reinterpret_cast<const float4*>(smem + kOffHdr + ib * kHdr);
-      if (K > 0)
+      // The lists carry over between consecutive items of one query block: an
+      // item's list then also holds earlier ranges' entries (the final merge
+      // skips repeats), and the carried k-th best filters this range early.
+      if (K > 0 && qb != prev_qb) {
         for (int e = t_id; e < kQB * kMaxTopk; e += kGroup) {
           top_s[e] = -INFINITY;
           top_i[e] = kNoIndex;
         }
+        if (t_id < kQB) {
+          thr_s[t_id] = -INFINITY;
+          thr_i[t_id] = kNoIndex;
+        }
+        if (!wsync()) { ok = false; break; }
+      }
+      prev_qb = qb;
       for (int64_t g = 0; ok && g < groups; ++g, ++gc) {
         const int64_t v = v0 + g * kGroup + t_id;
         const bool valid = v < v1;
@@ -538,7 +586,13 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(Args a) {
             const float Dm = comb(dm + 3 * qq), Ds = comb(ds + 3 * qq);
             const float sc = n * fmaf(rho, fmaf(c4.z, Ds, c4.w), fmaf(c4.x, Dm, c4.y));
             if (a.scores && valid && q < a.nq) a.scores[q * a.n_vec + v] = sc;
-            if (K > 0) cand[ql * kGroup + t_id] = valid ? sc : -INFINITY;
+            if (K > 0) {
+              // survivors: valid vectors ahead of the query's current k-th best
+              const bool sv = valid && better(sc, v, thr_s[ql], thr_i[ql]);
+              const uint32_t bits = __ballot_sync(0xffffffffu, sv);
+              if (sv) cand[ql * kGroup + t_id] = sc;
+              if (lane == 0) smask[ql * 8 + (t_id >> 5)] = bits;  // word = the warp's 32-vector block
+            }
           }
         }
         if (K == 0) continue;
@@ -549,49 +603,81 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(Args a) {
         for (int ql = wsel; ql < kQB; ql += 8) {
           float* ts = top_s + ql * kMaxTopk;
           int64_t* ti = top_i + ql * kMaxTopk;
-          const float thr_s = ts[K - 1];
-          const int64_t thr_i = ti[K - 1];
-          float cs[9];
-          int64_t ci[9];
-          bool any = false;
+          const uint32_t mw = lane < 8 ? smask[ql * 8 + lane] : 0u;
+          const int nsurv = __reduce_add_sync(0xffffffffu, (unsigned)__popc(mw));
+          if (nsurv == 0) continue;
+          // the list, lane r < K holding rank r
+          float ls = lane < K ? ts[lane] : -INFINITY;
+          int64_t li = lane < K ? ti[lane] : kNoIndex;
+          if (nsurv <= 24) {
+            // few survivors: insert each one that still beats the k-th best
+            float ks = __shfl_sync(0xffffffffu, ls, K - 1);
+            int64_t ki = __shfl_sync(0xffffffffu, li, K - 1);
+            for (int w8 = 0; w8 < 8; ++w8) {
+              uint32_t bits = __shfl_sync(0xffffffffu, mw, w8);
+              while (bits) {
+                const int t = 32 * w8 + __ffs(bits) - 1;
+                bits &= bits - 1;
+                const float cs = cand[ql * kGroup + t];
+                const int64_t ci = gbase + t;
+                if (!better(cs, ci, ks, ki)) continue;
+                const int pos = __popc(__ballot_sync(0xffffffffu, lane < K && better(ls, li, cs, ci)));
+                const float us = __shfl_up_sync(0xffffffffu, ls, 1);
+                const int64_t ui = __shfl_up_sync(0xffffffffu, li, 1);
+                if (lane == pos) {
+                  ls = cs;
+                  li = ci;
+                } else if (lane > pos) {
+                  ls = us;
+                  li = ui;
+                }
+                ks = __shfl_sync(0xffffffffu, ls, K - 1);
+                ki = __shfl_sync(0xffffffffu, li, K - 1);
+              }
+            }
+          } else {
+            // many survivors: K rounds of the warp's best over the survivors
+            // (8 per lane) and the list
+            float cs[9];
+            int64_t ci[9];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int t = lane + 32 * e;
-            cs[e] = cand[ql * kGroup + t];
-            ci[e] = gbase + t < v1 ? gbase + t : kNoIndex;
-            if (!better(cs[e], ci[e], thr_s, thr_i)) {
-              cs[e] = -INFINITY;
-              ci[e] = kNoIndex;
-            } else {
-              any = true;
+            for (int e = 0; e < 8; ++e) {
+              const int t = lane + 32 * e;
+              const bool sv = (__shfl_sync(0xffffffffu, mw, e) >> lane) & 1u;
+              cs[e] = sv ? cand[ql * kGroup + t] : -INFINITY;
+              ci[e] = sv ? gbase + t : kNoIndex;
+            }
+            cs[8] = ls;
+            ci[8] = li;
+            for (int r = 0; r < K; ++r) {
+              float bs = -INFINITY;
+              int64_t bi = kNoIndex;
+#pragma unroll
+              for (int e = 0; e < 9; ++e)
+                if (better(cs[e], ci[e], bs, bi)) {
+                  bs = cs[e];
+                  bi = ci[e];
+                }
+              warp_best(bs, bi);
+#pragma unroll
+              for (int e = 0; e < 9; ++e)
+                if (ci[e] == bi && cs[e] == bs) {
+                  cs[e] = -INFINITY;
+                  ci[e] = kNoIndex;
+                }
+              if (lane == r) {
+                ls = bs;
+                li = bi;
+              }
             }
           }
-          if (!__any_sync(0xffffffffu, any)) continue;
-          cs[8] = lane < K ? ts[lane] : -INFINITY;
-          ci[8] = lane < K ? ti[lane] : kNoIndex;
-          __syncwarp();
-          for (int r = 0; r < K; ++r) {
-            float bs = -INFINITY;
-            int64_t bi = kNoIndex;
-#pragma unroll
-            for (int e = 0; e < 9; ++e)
-              if (better(cs[e], ci[e], bs, bi)) {
-                bs = cs[e];
-                bi = ci[e];
-              }
-            float ws_ = bs;
-            int64_t wi = bi;
-            warp_best(ws_, wi);
-#pragma unroll
-            for (int e = 0; e < 9; ++e)
-              if (ci[e] == wi && cs[e] == ws_) {
-                cs[e] = -INFINITY;
-                ci[e] = kNoIndex;
-              }
-            if (lane == 0) {
-              ts[r] = ws_;
-              ti[r] = wi;
-            }
+          if (lane < K) {
+            ts[lane] = ls;
+            ti[lane] = li;
+          }
+          if (lane == K - 1) {
+            thr_s[ql] = ls;
+            thr_i[ql] = li;
           }
           __syncwarp();
         }
@@ -605,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) score_kernel(Args a) {
           a.cand_s[base + e] = top_s[ql * kMaxTopk + r];
           a.cand_i[base + e] = top_i[ql * kMaxTopk + r];
         }
-        if (!wsync()) { ok = false; break; }  // the lists are reset by the next item
+        if (!wsync()) { ok = false; break; }  // the next item resets or extends the lists
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(B(bar_hempty[ib]));
@@ -704,7 +790,7 @@ size_t workspace_bytes(const QParams& kp, int64_t nq, int64_t n_vec, int topk) {
   // the item count depends on the SM count: size the candidates for up to
   // 4 x 1024 items per query block
   const int64_t items_max = n_qb * std::min<int64_t>((n_vec + kGroup - 1) / kGroup, 4096);
-  size_t b = up256((size_t)n_qb * a.img_bytes);
+  size_t b = up256((size_t)n_qb * a.img_bytes) + up256((size_t)n_qb * kQB * 2 * 4);
   if (topk > 0) b += up256((size_t)items_max * kQB * topk * 4) + up256((size_t)items_max * kQB * topk * 8);
   return b;
 }
@@ -718,6 +804,8 @@ cudaError_t launch(const QParams& kp, const float* qrot, const float* u, int64_t
   unsigned char* w = (unsigned char*)ws;
   unsigned char* images = w;
   w += up256((size_t)n_qb * a.img_bytes);
+  float* qinv = (float*)w;
+  w += up256((size_t)n_qb * kQB * 2 * 4);
   a.codes = codes;
   a.signs = signs;
   a.norms = norms;
@@ -735,7 +823,11 @@ cudaError_t launch(const QParams& kp, const float* qrot, const float* u, int64_t
   }
   float alpha[8], asum;
   attn::odd_feature_coefs(kp.centroids, kp.k, alpha, &asum);
-  query_image_kernel<<<(unsigned)n_qb, 256, 0, st>>>(kp, a, alpha[0], alpha[1], alpha[2], alpha[3], qrot, u, images);
+  query_scale_kernel<<<(unsigned)((n_qb * kQB * 2 + 7) / 8), 256, 0, st>>>(kp, a, alpha[0], alpha[1], alpha[2],
+                                                                             alpha[3], qrot, u, qinv, images, n_qb);
+  const int kt4 = (a.fk * a.wpp + a.sw) * 8;
+  query_digits_kernel<<<dim3((unsigned)((kQB * kt4 + 255) / 256), (unsigned)n_qb), 256, 0, st>>>(
+      kp, a, alpha[0], alpha[1], alpha[2], alpha[3], qrot, u, qinv, images);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // one CTA per SM (it allocates all 512 TMEM columns): the shared memory

@@ -47,37 +47,6 @@ __global__ void __launch_bounds__(128) query_prep_hadamard_kernel(QParams qp,
   }
 }
 
-// Dense rotation: q' = Pi q, u = S q' (one warp per query; d <= 1536).
-__global__ void __launch_bounds__(128) query_prep_dense_kernel(QParams qp,
-                                                               const float* __restrict__ q,
-                                                               int64_t nq, int64_t ldq,
-                                                               float* __restrict__ qrot,
-                                                               float* __restrict__ u) {
-  extern __shared__ float dyn[];
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int64_t w = (int64_t)blockIdx.x * 4 + wib;
-  float* qs = dyn + wib * 2 * qp.d;
-  float* ps = qs + qp.d;
-  if (w >= nq) return;
-  for (int j = lane; j < qp.d; j += 32) qs[j] = q[w * ldq + j];
-  __syncwarp();
-  for (int i = lane; i < qp.d; i += 32) {
-    const float* row = qp.Pi + (size_t)i * qp.d;
-    float acc = 0.f;
-    for (int j = 0; j < qp.d; ++j) acc = fmaf(__ldg(row + j), qs[j], acc);
-    qrot[w * qp.d + i] = acc;
-    ps[i] = acc;
-  }
-  __syncwarp();
-  if (u) {
-    for (int i = lane; i < qp.m; i += 32) {
-      float acc = 0.f;
-      for (int j = 0; j < qp.d; ++j) acc = fmaf(__ldg(qp.St + (size_t)j * qp.m + i), ps[j], acc);
-      u[w * qp.m + i] = acc;
-    }
-  }
-}
-
 // scores[a][t] for a tile of QT queries (q' and u staged in shared memory)
 // and 128 vectors per CTA (one thread per vector).
 constexpr int kScoreThreads = 128;
