@@ -64,11 +64,12 @@ __device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
                : "memory");
 }
 
-// Bounded wait for the phase with the given parity (non-blocking polls:
-// measured faster here than a suspending try_wait): false, and the device
-// error word set, if it has not completed within the wait budget.
+// Bounded wait for the phase with the given parity (try_wait, which parks
+// the polling warp between tests and leaves its issue slots to the working
+// warps; measured slightly faster here than non-blocking polls): false, and
+// the device error word set, if it has not completed within the wait budget.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err) {
-  return bounded_wait<false>(bar, parity, err);
+  return bounded_wait<true>(bar, parity, err);
 }
 
 // Warp-uniform form: every lane waits, the warp proceeds only if all saw it.
