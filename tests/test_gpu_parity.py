@@ -275,6 +275,52 @@ def test_attention_end_to_end_qwen_shape_subset():
 # ------------------------------------------------------------------ dense rotation
 
 
+@pytest.mark.parametrize("d,m,bits,prod,dtype,layout,n,seg,cap", [
+    (256, 0, 3, False, "float16", tq.LAYOUT_ROW, 1000, 0, 0),
+    (256, 0, 2, False, "float32", tq.LAYOUT_BLOCK32, 288, 96, 128),    # 3 segments with a spare block each
+    (256, 512, 3, True, "bfloat16", tq.LAYOUT_ROW, 700, 0, 0),         # m = 2 d
+    (512, 256, 2, True, "float32", tq.LAYOUT_ROW, 450, 150, 160),      # m = d / 2, 3 segments
+])
+def test_dense_tensor_core_encode(d, m, bits, prod, dtype, layout, n, seg, cap):
+    # d and m multiples of 256 run the split-precision tensor-core products;
+    # ragged row counts leave a partial last tile of 128 rows
+    ora, lib = make_pair(d, bits, prod, seed=60 + d + bits, m=m if prod else None, dense=True)
+    x = synth.gaussian_vectors(n, d, seed=61, dtype=dtype, device=DEV, n_outliers=4, outlier_scale=20.0)
+    x[7] = 0  # a zero vector
+    seg = seg or n
+    cap = cap or seg
+    ns = n // seg
+    lay = "row" if layout == tq.LAYOUT_ROW else "block32"
+    if prod:
+        codes, signs, norms, rnorms = tq.tq_encode_prod(lib, x, seg_len=seg, seg_cap=cap)
+    else:
+        codes, norms = tq.tq_encode_mse(lib, x, layout=layout, seg_len=seg, seg_cap=cap)
+    torch.cuda.synchronize()
+    tq.tq_sync_check()
+    wc = u32(codes)
+    for s_ in range(ns):
+        xs = x_np(x[seg * s_:seg * (s_ + 1)])
+        e = ora.encode(xs, layout=lay)
+        if layout == tq.LAYOUT_ROW:
+            gi = o.unpack_row(wc[cap * s_:cap * s_ + seg], ora.k, ora.d_pad)
+        else:
+            blocks = cap // 32
+            gi = o.unpack_block32(wc[blocks * s_:blocks * (s_ + 1)], ora.k, ora.d_pad, seg)
+        _, bad = check_codes(gi, e["idx"], e["y"], ora.boundaries, ora.d_pad)
+        gn = norms.cpu().numpy()[cap * s_:cap * s_ + seg]
+        assert_close_rel(gn, e["norms"], 1e-30, what="norms")
+        if cap > seg:
+            assert np.all(norms.cpu().numpy()[cap * s_ + seg:cap * (s_ + 1)] == 0)
+        if prod:
+            nsg = check_signs(u32(signs)[cap * s_:cap * s_ + seg], e["signs"], e["z"], e["rho64"], m,
+                              skip_rows=bad)
+            assert nsg <= 1e-4 * seg * m
+            gr = rnorms.cpu().numpy()[cap * s_:cap * s_ + seg]
+            assert_close_rel(gr, e["rnorms"], 1e-30, what="rnorms", mask=~bad)
+    assert norms.cpu().numpy()[7] == 0.0
+
+
+
 @pytest.mark.parametrize("bits", [2, 4])
 def test_dense_rotation_encode_scores(bits):
     d = 256

@@ -16,6 +16,7 @@
 #include "tq_enc2_launch.h"
 #include "tq_enc3.h"
 #include "tq_gemm.cuh"
+#include "tq_gemm_tc.h"
 #include "tq_internal.h"
 #include "tq_score_tc.h"
 #include "tq_scores.cuh"
@@ -138,6 +139,75 @@ cudaError_t encode_dense(const QParams& qp, bool prod, const T* x, int64_t ld, i
 
 constexpr int64_t kDenseChunk = 32768;
 
+// The dense path on the tensor cores (split-precision products, see
+// tq_gemm_tc.h): y = Pi x as three fp16 terms, z = S r as two; the other
+// steps are the kernels above.  Covers d and m multiples of 128.
+bool dense_tc_covers(const QParams& qp, bool prod) {
+  return qp.rot == TQ_ROT_DENSE && qp.Pi2 && gemm_tc::covers(qp.d, qp.d) &&
+         (!prod || (qp.S16 && gemm_tc::covers(qp.m, qp.d)));
+}
+
+cudaError_t encode_dense_tc(const QParams& qp, bool prod, const void* x, int dt, int64_t ld, int64_t n_vec,
+                            int64_t seg_len, int64_t seg_cap, int layout, uint32_t* codes, uint32_t* signs,
+                            float* norms, float* rnorms, float* ws, int64_t chunk, cudaStream_t st) {
+  const int d = qp.d;
+  uint16_t* a2 = reinterpret_cast<uint16_t*>(ws);  // [chunk][2 d] fp16: x, then r
+  float* y = ws + (size_t)chunk * d;                // [chunk][d]  (y, then r)
+  float* z = y + (size_t)chunk * d;                 // [chunk][m]
+  unsigned* err = device_error_ptr();
+  const int nsm = num_sms();
+  int64_t row = 0;
+  while (row < n_vec) {
+    // a chunk never crosses a segment boundary and starts on a 32-block
+    const int64_t t = row % seg_len;
+    const int64_t rows = std::min<int64_t>(chunk, seg_len - t);
+    cudaError_t e = gemm_tc::prep_rows(dt, x, ld, d, seg_len, seg_cap, row, rows, a2, norms, st);
+    if (e != cudaSuccess) return e;
+    gemm_tc::Problem g1{};
+    g1.A = a2;
+    g1.lda = 2 * d;
+    g1.M = rows;
+    g1.B = qp.Pi2;
+    g1.ldb = 2 * d;
+    g1.N = d;
+    g1.K = d;
+    g1.nterms = 3;  // hi.lo + lo.hi + hi.hi (the small terms first)
+    g1.a_off[0] = 0, g1.b_off[0] = d;
+    g1.a_off[1] = d, g1.b_off[1] = 0;
+    g1.a_off[2] = 0, g1.b_off[2] = 0;
+    g1.scale = 1.0f / (gemm_tc::kSplitScale * gemm_tc::kSplitScale);
+    g1.C = y;
+    g1.ldc = d;
+    e = gemm_tc::run(g1, err, nsm, st);
+    if (e != cudaSuccess) return e;
+    quantize_rows_kernel<<<(unsigned)ceil_div(ceil_div(rows, 32), 4), 128, 0, st>>>(
+        qp, y, seg_len, seg_cap, row, rows, layout, prod, codes, norms, rnorms);
+    if (prod) {
+      e = gemm_tc::split_rows(y, d, rows, a2, st);
+      if (e != cudaSuccess) return e;
+      gemm_tc::Problem g2{};
+      g2.A = a2;
+      g2.lda = 2 * d;
+      g2.M = rows;
+      g2.B = qp.S16;  // exact in fp16
+      g2.ldb = d;
+      g2.N = qp.m;
+      g2.K = d;
+      g2.nterms = 2;  // lo.S + hi.S (the small term first)
+      g2.a_off[0] = d, g2.b_off[0] = 0;
+      g2.a_off[1] = 0, g2.b_off[1] = 0;
+      g2.scale = 1.0f / gemm_tc::kSplitScale;
+      g2.C = z;
+      g2.ldc = qp.m;
+      e = gemm_tc::run(g2, err, nsm, st);
+      if (e != cudaSuccess) return e;
+      pack_signs_kernel<<<(unsigned)ceil_div(rows, 4), 128, 0, st>>>(z, qp.m, seg_len, seg_cap, row, rows, signs);
+    }
+    row += rows;
+  }
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------- thread-per-vector encode
 
 // Returns true (and launches) when the thread-per-vector kernels cover the
@@ -240,6 +310,9 @@ int launch_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n
   if (qp.rot == TQ_ROT_DENSE) {
     const int64_t chunk = std::min<int64_t>(kDenseChunk, round_up(n_vec, 32));
     float* w = (float*)ws;
+    if (dense_tc_covers(qp, prod))
+      return encode_dense_tc(qp, prod, x, dt, ld, n_vec, seg_len, seg_cap, layout, codes, signs, norms, rnorms, w,
+                             chunk, st);
     switch (dt) {
       case TQ_F32: return encode_dense(qp, prod, (const float*)x, ld, n_vec, seg_len, seg_cap, layout, codes, signs, norms, rnorms, w, chunk, st);
       case TQ_F16: return encode_dense(qp, prod, (const __half*)x, ld, n_vec, seg_len, seg_cap, layout, codes, signs, norms, rnorms, w, chunk, st);

@@ -15,6 +15,7 @@
 #include <mutex>
 #include <vector>
 
+#include "tq_gemm_tc.h"
 #include "tq_internal.h"
 
 namespace tq {
@@ -278,6 +279,7 @@ tq_status tq_params_destroy(tq_params* p) {
   cudaFree(p->dev_St);
   cudaFree(p->dev_S16);
   cudaFree(p->dev_Pi);
+  cudaFree(p->dev_Pi2);
   cudaSetDevice(cur);
   std::free(p->host_Pi);
   delete p;
@@ -394,6 +396,13 @@ tq_status tq_params_create(int d, int bits, tq_mode mode, tq_rot rot, int m, con
     if (cudaMemcpy(p->dev_Pi, p->host_Pi, n * 4, cudaMemcpyHostToDevice) != cudaSuccess)
       return fail(TQ_ERR_CUDA);
     q.Pi = (const float*)p->dev_Pi;
+    // the tensor-core encoder's operand: [hi | lo] fp16 of 2^8 Pi
+    std::vector<uint16_t> pi2(2 * n);
+    tq::gemm_tc::split_host(p->host_Pi, d, d, pi2.data());
+    if (cudaMalloc(&p->dev_Pi2, 2 * n * 2) != cudaSuccess) return fail(TQ_ERR_CUDA);
+    if (cudaMemcpy(p->dev_Pi2, pi2.data(), 2 * n * 2, cudaMemcpyHostToDevice) != cudaSuccess)
+      return fail(TQ_ERR_CUDA);
+    q.Pi2 = (const uint16_t*)p->dev_Pi2;
   }
   (void)st;
   *out = p;

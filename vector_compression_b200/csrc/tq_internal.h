@@ -32,6 +32,7 @@ struct QParams {
   const float* St;     // device [d_pad][m] fp32 (S transposed)
   const uint16_t* S16; // device [m][d_pad] fp16 bits
   const float* Pi;     // device [d][d] fp32 (DENSE), y = Pi x
+  const uint16_t* Pi2; // device [d][2 d] fp16 bits (DENSE): [hi | lo] of 2^8 Pi
 };
 
 }  // namespace tq
@@ -45,6 +46,7 @@ struct tq_params {
   void* dev_St;
   void* dev_S16;
   void* dev_Pi;
+  void* dev_Pi2;
   float host_centroids[tq::kMaxLevels];
   float host_boundaries[tq::kMaxLevels];
   float* host_Pi;      // d*d, DENSE only
