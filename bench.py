@@ -54,6 +54,9 @@ def parse():
                     help="instead of the KV-cache step, time the retrieval set (1e6 x 1536 unit vectors, dense "
                          "rotation): Q_prod encode of the whole set and scores + top-10 for this many queries")
     ap.add_argument("--retrieval-bits", type=int, default=2, choices=[2, 4])
+    ap.add_argument("--retrieval-vectors", type=int, default=0,
+                    help="size of the retrieval set (0 = the 1e6 of the workload; smaller sets are for profiler "
+                         "captures)")
     ap.add_argument("--qjl-rows", type=int, default=0,
                     help="QJL projection rows m of the keys (0 = the padded head dim; d_pad / 2 is the half-size variant)")
     return ap.parse_args()
@@ -246,7 +249,7 @@ def run_retrieval(args):
     import vector_compression_b200 as tq
 
     R = synth.RETRIEVAL
-    n, d, m, bits = R["n"], R["d"], R["m"], args.retrieval_bits
+    n, d, m, bits = args.retrieval_vectors or R["n"], R["d"], R["m"], args.retrieval_bits
     dr = synth.method_draws(d, m, R["seed"], dense=True)
     p = tq.TQParams(d, bits, tq.MODE_PROD, tq.ROT_DENSE, m=m, S=dr["S"], G=dr["G"])
     dev = torch.device("cuda", 0)
@@ -284,7 +287,8 @@ def run_retrieval(args):
     peak_tf = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] \
         if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1590.0
     line = {
-        "metric": "retrieval set: Q_prod encode and scores + top-10", "workload": "retrieval 1e6 x 1536, dense",
+        "metric": "retrieval set: Q_prod encode and scores + top-10",
+        "workload": f"retrieval {'1e6' if n == 1_000_000 else n} x {d}, dense",
         "bits": bits, "m": m, "queries": nq,
         "encode": {"ms": enc_ms, "GB/s": enc_bytes / (enc_ms * 1e-3) / 1e9,
                    "TFLOP/s": enc_flop / (enc_ms * 1e-3) / 1e12,
@@ -293,7 +297,9 @@ def run_retrieval(args):
                         "frac_of_bf16_peak": sc_flop / (sc_ms * 1e-3) / 1e12 / peak_tf,
                         "pairs_per_s": nq * n / (sc_ms * 1e-3)},
         "recall_at_10": recall,
-        "arithmetic": {"encode": "fp32 GEMMs for Pi x and S r",
+        "arithmetic": {"encode": "Pi x and S r as tcgen05 fp16 contractions of split operands (hi.lo + lo.hi + "
+                                 "hi.hi and lo.S + hi.S, operands split into fp16 hi + lo), fp32 accumulation per "
+                                 "128-wide K chunk, chunk sums added in fp32",
                        "scores": "exact integer tcgen05 contractions of the code and sign bits against 24-bit "
                                  "fixed-point q' and S q'; fused per-query top-10"},
         "peak": "measured bf16 tensor figure (algorithmic flop: 2 d^2 + 2 m d per encoded vector, "

@@ -123,8 +123,11 @@ cudaError_t encode_dense(const QParams& qp, bool prod, const T* x, int64_t ld, i
         x, ld, d, seg_len, seg_cap, row, rows, xh, norms);
     cudaError_t e = gemm_abt_f32(xh, qp.Pi, y, (int)rows, d, d, st);
     if (e != cudaSuccess) return e;
-    quantize_rows_kernel<<<(unsigned)ceil_div(ceil_div(rows, 32), 4), 128, 0, st>>>(
-        qp, y, seg_len, seg_cap, row, rows, layout, prod, codes, norms, rnorms);
+    if (layout == TQ_LAYOUT_ROW)
+      launch_quantize_rows_warp(qp, y, seg_len, seg_cap, row, rows, prod, codes, norms, rnorms, st);
+    else
+      quantize_rows_kernel<<<(unsigned)ceil_div(ceil_div(rows, 32), 4), 128, 0, st>>>(
+          qp, y, seg_len, seg_cap, row, rows, layout, prod, codes, norms, rnorms);
     if (prod) {
       e = gemm_abt_f32(y, qp.S, z, (int)rows, qp.m, d, st);
       if (e != cudaSuccess) return e;
@@ -180,8 +183,11 @@ cudaError_t encode_dense_tc(const QParams& qp, bool prod, const void* x, int dt,
     g1.ldc = d;
     e = gemm_tc::run(g1, err, nsm, st);
     if (e != cudaSuccess) return e;
-    quantize_rows_kernel<<<(unsigned)ceil_div(ceil_div(rows, 32), 4), 128, 0, st>>>(
-        qp, y, seg_len, seg_cap, row, rows, layout, prod, codes, norms, rnorms);
+    if (layout == TQ_LAYOUT_ROW)
+      launch_quantize_rows_warp(qp, y, seg_len, seg_cap, row, rows, prod, codes, norms, rnorms, st);
+    else
+      quantize_rows_kernel<<<(unsigned)ceil_div(ceil_div(rows, 32), 4), 128, 0, st>>>(
+          qp, y, seg_len, seg_cap, row, rows, layout, prod, codes, norms, rnorms);
     if (prod) {
       e = gemm_tc::split_rows(y, d, rows, a2, st);
       if (e != cudaSuccess) return e;

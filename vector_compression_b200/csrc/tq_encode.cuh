@@ -277,6 +277,77 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(
   }
 }
 
+// Dense path, step 3 for ROW codes: one warp per row, the word positions of
+// a row independent of each other so that their loads are in flight
+// together (the task-per-32-rows kernel above walks them one by one).  Same
+// arithmetic and order as that kernel: idx = #{B_k < y}, code word p * A + a
+// = the ballot of bit p, and for Q_prod r = y - C[idx] over y with
+// rho = ||r||; the unbiased Q_MSE divides the norm by <y, C[idx]>.
+template <int K>
+__global__ void __launch_bounds__(256) quantize_rows_warp_kernel(
+    QParams qp, float* __restrict__ y, int64_t seg_len, int64_t seg_cap, int64_t row0, int64_t nrows, bool prod,
+    uint32_t* __restrict__ codes, float* __restrict__ norms, float* __restrict__ rnorms) {
+  __shared__ SmemCodebook cb;
+  load_codebook(cb, qp);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (w >= nrows) return;
+  constexpr int k = K, nb = (1 << K) - 1;
+  const int A = qp.d_pad / 32, d = qp.d;
+  const int64_t row = row0 + w;
+  const int64_t slot = (row / seg_len) * seg_cap + row % seg_len;
+  float* yr = y + w * (int64_t)d;
+  uint32_t* cw = codes + slot * qp.code_words;
+  float rr = 0.f, dot = 0.f;
+#pragma unroll 4
+  for (int a = 0; a < A; ++a) {
+    const float v = yr[32 * a + lane];
+    int idx = 0;  // #{B_j < v}, as quantize_index
+#pragma unroll
+    for (int j = 0; j < nb; ++j) idx += (cb.b[j] < v) ? 1 : 0;
+    const float c = cb.c[idx];
+    dot = fmaf(v, c, dot);
+#pragma unroll
+    for (int p = 0; p < k; ++p) {
+      const uint32_t word = __ballot_sync(0xffffffffu, (idx >> p) & 1);
+      if (lane == p) cw[p * A + a] = word;
+    }
+    if (prod) {
+      const float r = v - c;
+      rr = fmaf(r, r, rr);
+      yr[32 * a + lane] = r;
+    }
+  }
+  if (prod) {
+    rr = warp_sum(rr);
+    if (lane == 0) put_rnorm(rnorms, slot, sqrtf(rr), qp.rnorm_f16);
+  } else if (qp.unbiased) {  // EDEN's scale n / <y, C[idx]>
+    dot = warp_sum(dot);
+    if (lane == 0) norms[slot] = dot > 0.f ? norms[slot] / dot : 0.f;
+  }
+}
+
+inline void launch_quantize_rows_warp(const QParams& qp, float* y, int64_t seg_len, int64_t seg_cap, int64_t row0,
+                                      int64_t nrows, bool prod, uint32_t* codes, float* norms, float* rnorms,
+                                      cudaStream_t st) {
+  const unsigned blocks = (unsigned)ceil_div(nrows, 8);
+  switch (qp.k) {
+#define TQ_QRW(KK)                                                                                       \
+  case KK:                                                                                              \
+    quantize_rows_warp_kernel<KK><<<blocks, 256, 0, st>>>(qp, y, seg_len, seg_cap, row0, nrows, prod,  \
+                                                            codes, norms, rnorms);                      \
+    break;
+    TQ_QRW(1)
+    TQ_QRW(2)
+    TQ_QRW(3)
+    TQ_QRW(4)
+#undef TQ_QRW
+    default:
+      break;
+  }
+}
+
 // Dense path, step 5: sign bits of z = r S^T (fp32 [nrows][m]).
 __global__ void __launch_bounds__(128) pack_signs_kernel(const float* __restrict__ z, int m,
                                                          int64_t seg_len, int64_t seg_cap,

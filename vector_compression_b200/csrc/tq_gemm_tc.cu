@@ -4,16 +4,19 @@
 // A persistent CTA per SM walks the output tiles of 128 x 128 (tile t: row
 // block t / (N / 128), column block t % (N / 128), so CTAs that run at the
 // same time share row blocks of A in L2, and B stays in L2).  K is taken in
-// chunks of 128 columns; a chunk's MMAs (every term, in the given order)
+// chunks of 64 columns; a chunk's MMAs (every term, in the given order)
 // accumulate into one of four 128-column TMEM accumulators.
-//   warp 0      TMA producer: per pipeline stage a 128 x 64 box of A and of B
-//               (128-byte swizzle), 6-stage ring;
+//   warp 0      TMA producer: per pipeline stage the 128 x 64 boxes (128-byte
+//               swizzle) of the chunk's distinct A and B column ranges, each
+//               loaded once however many terms read it, in a ring of as
+//               many stages as 192 KB holds (3 for four boxes, 4 for three);
 //   warp 1      TMEM allocator (512 columns) and MMA issuer: tcgen05.mma
 //               kind::f16 (M 128, N 128, K 16), fp32 accumulation;
-//   warps 2..5  epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (its 32
-//               rows), adds each chunk's sums into the row's 128 fp32
-//               registers (round to nearest), releases the accumulator, and
-//               after the last chunk stores the scaled row.
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (its 32
+//               rows), columns 64 h .. 64 h + 63 with h = (w - 2) / 4, adds
+//               each chunk's sums into 64 fp32 registers per row (round to
+//               nearest), releases the accumulator, and after the last chunk
+//               stores its 64 scaled values of the row.
 // Every wait is bounded (device error word + clean exit).
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -31,18 +34,24 @@ namespace gemm_tc {
 
 namespace {
 
-constexpr int kStages = 6;
+constexpr int kMaxStages = 6;
 constexpr int kAcc = 4;  // chunk accumulators in TMEM
-constexpr int kThreads = 192;
-constexpr uint32_t kABytes = kBM * kBK * 2;         // 16 KB
-constexpr uint32_t kBBytes = kBN * kBK * 2;         // 16 KB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;  // 32 KB (a multiple of 1024)
-constexpr uint32_t kSmem = kStages * kStageBytes + 1024;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kMaxBoxes = 4;                              // distinct A + B ranges per stage
+constexpr uint32_t kBoxBytes = kBM * kBK * 2;              // 16 KB (kBM == kBN)
+constexpr uint32_t kRing = 192 * 1024;                     // stage ring bytes
+constexpr uint32_t kSmem = kRing + 1024;
+static_assert(kBM == kBN && kKC == kBK, "one box size, one stage per chunk");
 
 struct Args {
   int64_t M;
   int N, K, nterms;
-  int a_off0, a_off1, a_off2, b_off0, b_off1, b_off2;
+  int na, nb;                   // distinct A and B column ranges
+  int a_base0, a_base1, a_base2;  // their first columns
+  int b_base0, b_base1, b_base2;
+  int ia0, ia1, ia2, ib0, ib1, ib2;  // term t reads A box ia_t and B box ib_t
+  int stages;                        // ring stages of (na + nb) boxes
   float scale;
   float* C;
   int64_t ldc;
@@ -93,20 +102,23 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
   return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
-// 32 columns of this warp's 32 TMEM lanes, load and completion in one
-// statement (the registers are defined once the data has arrived)
-__device__ __forceinline__ void tmem_ld32_sync(uint32_t addr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
         "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
         "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
         "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(addr)
-      : "memory");
+      : "r"(addr));
+}
+// completes this thread's outstanding tcgen05.ld; the empty statements keep
+// every use of the registers after the wait
+__device__ __forceinline__ void tmem_ld_wait2(uint32_t (&r)[32], uint32_t (&q)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]), "+r"(q[i]));
 }
 
 __device__ __forceinline__ int pick(int t, int v0, int v1, int v2) { return t == 0 ? v0 : (t == 1 ? v1 : v2); }
@@ -114,18 +126,19 @@ __device__ __forceinline__ int pick(int t, int v0, int v1, int v2) { return t ==
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap, Args a) {
   extern __shared__ unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t bar_full[kStages], bar_empty[kStages], bar_pfull[kAcc], bar_pempty[kAcc], bar_done;
+  __shared__ __align__(8) uint64_t bar_full[kMaxStages], bar_empty[kMaxStages], bar_pfull[kAcc], bar_pempty[kAcc],
+      bar_done;
   __shared__ uint32_t tmem_base_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < a.stages; ++s) {
       mbar_init(smem_u32(&bar_full[s]), 1);
       mbar_init(smem_u32(&bar_empty[s]), 1);
     }
     for (int b = 0; b < kAcc; ++b) {
       mbar_init(smem_u32(&bar_pfull[b]), 1);
-      mbar_init(smem_u32(&bar_pempty[b]), 4);  // one arrival per epilogue warp
+      mbar_init(smem_u32(&bar_pempty[b]), kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(smem_u32(&bar_done), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -139,8 +152,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
-  const int n_chunks = a.K / kKC;                 // K chunks per tile
-  const int kb_chunk = a.nterms * (kKC / kBK);    // pipeline stages per chunk
+  const int n_chunks = a.K / kKC;  // K chunks (= pipeline stages) per tile
+  const uint32_t nst = (uint32_t)a.stages, stage_bytes = (uint32_t)(a.na + a.nb) * kBoxBytes;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -149,24 +162,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int64_t tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x) {
         const int mb = (int)(tile / a.tiles_n), nb = (int)(tile % a.tiles_n);
-        for (int c = 0; ok && c < n_chunks; ++c)
-          for (int kk = 0; kk < kb_chunk; ++kk, ++it) {
-            const int t = kk / (kKC / kBK), k0 = c * kKC + (kk % (kKC / kBK)) * kBK;
-            const uint32_t s = it % kStages;
-            if (it >= (uint32_t)kStages && !wait_bar(smem_u32(&bar_empty[s]), ((it / kStages) - 1) & 1u, a.err)) {
-              ok = false;
-              break;
-            }
-            const uint32_t sa = smem_u32(smem + s * kStageBytes);
-            mbar_expect(smem_u32(&bar_full[s]), kStageBytes);
-            tma_load_2d(sa, &amap, pick(t, a.a_off0, a.a_off1, a.a_off2) + k0, mb * kBM, smem_u32(&bar_full[s]));
-            tma_load_2d(sa + kABytes, &bmap, pick(t, a.b_off0, a.b_off1, a.b_off2) + k0, nb * kBN,
-                        smem_u32(&bar_full[s]));
+        for (int c = 0; c < n_chunks; ++c, ++it) {
+          const uint32_t s = it % nst;
+          if (it >= nst && !wait_bar(smem_u32(&bar_empty[s]), ((it / nst) - 1) & 1u, a.err)) {
+            ok = false;
+            break;
           }
+          const uint32_t sa = smem_u32(smem + s * stage_bytes);
+          const uint32_t bar = smem_u32(&bar_full[s]);
+          mbar_expect(bar, (uint32_t)(a.na + a.nb) * kBoxBytes);
+          for (int i = 0; i < a.na; ++i)
+            tma_load_2d(sa + i * kBoxBytes, &amap, pick(i, a.a_base0, a.a_base1, a.a_base2) + c * kKC, mb * kBM, bar);
+          for (int j = 0; j < a.nb; ++j)
+            tma_load_2d(sa + (a.na + j) * kBoxBytes, &bmap, pick(j, a.b_base0, a.b_base1, a.b_base2) + c * kKC,
+                        nb * kBN, bar);
+        }
       }
       // the CTA leaves no copy in flight
-      for (uint32_t c = it > (uint32_t)kStages ? it - kStages : 0; c < it; ++c)
-        wait_bar(smem_u32(&bar_full[c % kStages]), (c / kStages) & 1u, nullptr);
+      for (uint32_t c = it > nst ? it - nst : 0; c < it; ++c)
+        wait_bar(smem_u32(&bar_full[c % nst]), (c / nst) & 1u, nullptr);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -184,19 +198,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t d = tmem + pb * (uint32_t)kBN;
-          for (int kk = 0; kk < kb_chunk; ++kk, ++it) {
-            const uint32_t s = it % kStages;
-            if (!wait_bar(smem_u32(&bar_full[s]), (it / kStages) & 1u, a.err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t sa = smem_u32(smem + s * kStageBytes), sb = sa + kABytes;
+          const uint32_t s = it % nst;
+          if (!wait_bar(smem_u32(&bar_full[s]), (it / nst) & 1u, a.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * stage_bytes);
+          for (int t = 0; t < a.nterms; ++t) {
+            const uint32_t ab = sa + (uint32_t)pick(t, a.ia0, a.ia1, a.ia2) * kBoxBytes;
+            const uint32_t bb = sa + (uint32_t)(a.na + pick(t, a.ib0, a.ib1, a.ib2)) * kBoxBytes;
 #pragma unroll
             for (int k4 = 0; k4 < kBK / 16; ++k4)
-              mma_f16(d, desc_sw128(sa + 32u * k4), desc_sw128(sb + 32u * k4), idesc, (kk | k4) ? 1u : 0u);
-            tc_commit(smem_u32(&bar_empty[s]));
+              mma_f16(d, desc_sw128(ab + 32u * k4), desc_sw128(bb + 32u * k4), idesc, (t | k4) ? 1u : 0u);
           }
+          tc_commit(smem_u32(&bar_empty[s]));
+          ++it;
           if (!ok) break;
           tc_commit(smem_u32(&bar_pfull[pb]));
         }
@@ -207,15 +224,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;
+    const int q = warp & 3, h = (warp - 2) >> 2;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    constexpr int kCols = kBN / 2;  // columns per thread
     uint32_t gc = 0;
     bool ok = true;
     for (int64_t tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x) {
       const int mb = (int)(tile / a.tiles_n), nb = (int)(tile % a.tiles_n);
-      float acc[kBN];  // this row's sums over the chunks so far
+      float acc[kCols];  // this row's sums over the chunks so far
 #pragma unroll
-      for (int j = 0; j < kBN; ++j) acc[j] = 0.f;
+      for (int j = 0; j < kCols; ++j) acc[j] = 0.f;
       for (int c = 0; c < n_chunks; ++c, ++gc) {
         const uint32_t pb = gc % kAcc;
         if (!wait_bar_warp(smem_u32(&bar_pfull[pb]), (gc / kAcc) & 1u, a.err)) {
@@ -223,12 +241,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        uint32_t r0[32], r1[32];
+        const uint32_t col = tmem + pb * (uint32_t)kBN + lane_off + (uint32_t)(kCols * h);
+        tmem_ld32(col, r0);
+        tmem_ld32(col + 32u, r1);
+        tmem_ld_wait2(r0, r1);
 #pragma unroll
-        for (int j = 0; j < kBN / 32; ++j) {
-          uint32_t r[32];
-          tmem_ld32_sync(tmem + pb * (uint32_t)kBN + lane_off + 32u * j, r);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) acc[32 * j + i] += __uint_as_float(r[i]);
+        for (int i = 0; i < 32; ++i) {
+          acc[i] += __uint_as_float(r0[i]);
+          acc[32 + i] += __uint_as_float(r1[i]);
         }
         // the accumulator has been read: free for the chunk kAcc later
         tc_fence_before();
@@ -238,9 +259,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       const int64_t row = (int64_t)mb * kBM + 32 * q + lane;
       if (row < a.M) {
-        float4* dst = reinterpret_cast<float4*>(a.C + row * a.ldc + (int64_t)nb * kBN);
+        float4* dst = reinterpret_cast<float4*>(a.C + row * a.ldc + (int64_t)nb * kBN + kCols * h);
 #pragma unroll
-        for (int v = 0; v < kBN / 4; ++v)
+        for (int v = 0; v < kCols / 4; ++v)
           dst[v] = make_float4(a.scale * acc[4 * v], a.scale * acc[4 * v + 1], a.scale * acc[4 * v + 2],
                                a.scale * acc[4 * v + 3]);
       }
@@ -363,12 +384,31 @@ cudaError_t run(const Problem& p, unsigned* err, int num_sms, cudaStream_t st) {
   a.N = p.N;
   a.K = p.K;
   a.nterms = p.nterms;
-  a.a_off0 = p.a_off[0];
-  a.a_off1 = p.nterms > 1 ? p.a_off[1] : 0;
-  a.a_off2 = p.nterms > 2 ? p.a_off[2] : 0;
-  a.b_off0 = p.b_off[0];
-  a.b_off1 = p.nterms > 1 ? p.b_off[1] : 0;
-  a.b_off2 = p.nterms > 2 ? p.b_off[2] : 0;
+  // distinct column ranges of A and of B, and which box each term reads
+  int abase[3], bbase[3], ia[3] = {0, 0, 0}, ib[3] = {0, 0, 0};
+  int na = 0, nbx = 0;
+  for (int t = 0; t < p.nterms; ++t) {
+    int i = 0;
+    while (i < na && abase[i] != p.a_off[t]) ++i;
+    if (i == na) abase[na++] = p.a_off[t];
+    ia[t] = i;
+    int j = 0;
+    while (j < nbx && bbase[j] != p.b_off[t]) ++j;
+    if (j == nbx) bbase[nbx++] = p.b_off[t];
+    ib[t] = j;
+  }
+  if (na + nbx > kMaxBoxes) return cudaErrorInvalidValue;
+  a.stages = std::min<int>(kMaxStages, (int)(kRing / ((uint32_t)(na + nbx) * kBoxBytes)));
+  a.na = na;
+  a.nb = nbx;
+  a.a_base0 = abase[0];
+  a.a_base1 = na > 1 ? abase[1] : 0;
+  a.a_base2 = na > 2 ? abase[2] : 0;
+  a.b_base0 = bbase[0];
+  a.b_base1 = nbx > 1 ? bbase[1] : 0;
+  a.b_base2 = nbx > 2 ? bbase[2] : 0;
+  a.ia0 = ia[0], a.ia1 = ia[1], a.ia2 = ia[2];
+  a.ib0 = ib[0], a.ib1 = ib[1], a.ib2 = ib[2];
   a.scale = p.scale;
   a.C = p.C;
   a.ldc = p.ldc;

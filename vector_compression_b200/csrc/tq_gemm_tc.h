@@ -11,12 +11,13 @@
 // into one accumulator (measured here on B200: the error of y grows about
 // linearly with the chain length, as a truncating add would), and the QJL
 // signs amplify a relative error of y by |S y| / rho.  So every chunk of
-// kKC = 128 columns of K (all terms of the chunk, the small lo terms first)
+// kKC = 64 columns of K (all terms of the chunk, the small lo terms first)
 // accumulates into a fresh TMEM accumulator, and the chunk sums are added in
 // fp32 with round-to-nearest on the CUDA cores.  Measured at d = m = 1536
-// against fp64: y within 0.16 of the code window 1e-5 / sqrt(d), and z within
-// 0.63 of the sign window 1e-5 rho when formed from that y (a plain fp32
-// GEMM: 2.1), 0.13 for the z product itself.
+// against fp64 (chunks done as separate products): y within 0.11 of the code
+// window 1e-5 / sqrt(d) and z within 0.43 of the sign window 1e-5 rho when
+// formed from that y (one 288-MMA chain: 6.6 and more; a plain fp32 GEMM:
+// 1.1 and 2.1).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -31,7 +32,7 @@ namespace gemm_tc {
 constexpr int kBM = 128;  // rows per tile (MMA M)
 constexpr int kBN = 128;  // columns per tile (MMA N)
 constexpr int kBK = 64;   // K per pipeline stage (one 128-byte swizzle row of fp16)
-constexpr int kKC = 128;  // K per accumulation chunk (see below)
+constexpr int kKC = 64;   // K per accumulation chunk (see below)
 constexpr float kSplitScale = 256.0f;  // 2^8: keeps the lo parts of unit-scale rows normal in fp16
 
 // C[M][N] (fp32, row stride ldc) = scale * sum over terms t of
@@ -53,7 +54,8 @@ struct Problem {
   int64_t ldc;  // elements
 };
 
-// Shapes the kernel covers: N and K multiples of 128.
+// Shapes the kernel covers: N a multiple of 128, K a multiple of 64, at most
+// four distinct column ranges among the terms' A and B operands.
 bool covers(int N, int K);
 
 // Runs the product (persistent CTAs, at most num_sms); every wait in the
