@@ -368,7 +368,6 @@ int launch_decode(const QParams& qp, int layout, const uint32_t* codes, const ui
 int launch_query_prep(const QParams& qp, const float* q, int64_t nq, int64_t ldq, float* qrot,
                       float* u, void* stream) {
   cudaStream_t st = S(stream);
-  const unsigned blocks = (unsigned)ceil_div(nq, 4);
   if (nq == 0) return cudaSuccess;
   if (qp.rot == TQ_ROT_DENSE) {
     // q' = Pi q and u = S q' as tiled GEMMs over all queries (rows of up to
@@ -383,10 +382,18 @@ int launch_query_prep(const QParams& qp, const float* q, int64_t nq, int64_t ldq
     }
     return cudaSuccess;
   }
+  // one query per block while that leaves SMs idle, four (sharing the S^T
+  // loads) once there are many
+  const bool four = nq >= (int64_t)num_sms() * 4;
+  const unsigned qblocks = (unsigned)ceil_div(nq, four ? 4 : 1);
+  const unsigned qthreads = qp.m >= 256 ? 256 : 128;  // threads over the m outputs of u
   switch (qp.d_pad / 32) {
 #define TQ_QP(AA)                                                                                \
   case AA:                                                                                       \
-    query_prep_hadamard_kernel<AA><<<blocks, 128, 0, st>>>(qp, q, nq, ldq, qrot, u);             \
+    if (four)                                                                                    \
+      query_prep_hadamard_kernel<AA, 4><<<qblocks, qthreads, 0, st>>>(qp, q, nq, ldq, qrot, u);  \
+    else                                                                                         \
+      query_prep_hadamard_kernel<AA, 1><<<qblocks, qthreads, 0, st>>>(qp, q, nq, ldq, qrot, u);  \
     break;
     TQ_QP(1)
     TQ_QP(2)
@@ -440,8 +447,11 @@ size_t attention_workspace(const QParams& kp, const QParams& vp, int L, int B, i
   int64_t chunk = round_up(ceil_div(seq, n_chunks), 64);
   if (chunk < 1024) {
     // short chunks would spend most of a CTA on its per-query setup: aim at
-    // one wave of CTAs instead
-    n_chunks = std::max<int64_t>(1, (int64_t)num_sms() * 4 / std::max<int64_t>(groups, 1));
+    // one wave of CTAs instead (four per SM at d_pad 128; at d_pad 256, whose
+    // CTAs run one per SM, two, measured 8% faster than four on a 128K-token
+    // cache of 8 groups)
+    const int64_t per_sm = kp.d_pad > 128 ? 2 : 4;
+    n_chunks = std::max<int64_t>(1, (int64_t)num_sms() * per_sm / std::max<int64_t>(groups, 1));
     chunk = round_up(ceil_div(seq, n_chunks), 64);
   }
   chunk = std::max<int64_t>(chunk, 256);
@@ -532,11 +542,11 @@ int launch_decode_attention(const QParams& kp, const QParams& vp, const float* q
   cudaError_t ce = cudaGetLastError();
   if (ce != cudaSuccess) return ce;
   }
-  const unsigned cblocks = (unsigned)ceil_div((int64_t)sh.groups * sh.G, 4);
+  const unsigned cblocks = (unsigned)((int64_t)sh.groups * sh.G);  // one per (group, head)
   switch (vp.d_pad / 32) {
 #define TQ_CMB(AA)                                                                                 \
   case AA:                                                                                         \
-    attention_combine_hadamard_kernel<AA><<<cblocks, 128, 0, st>>>(vp, sh, part, out, Hq, Hkv);    \
+    attention_combine_hadamard_kernel<AA><<<cblocks, 256, 0, st>>>(vp, sh, part, out, Hq, Hkv);    \
     break;
     TQ_CMB(1)
     TQ_CMB(2)

@@ -187,28 +187,56 @@ __global__ void __launch_bounds__(kAttnThreads) attention_chunk_kernel(
 }
 
 // Merge chunk partials by log-sum-exp and apply Pi_V^T (Hadamard: D H / sqrt(d_pad)).
+// One block of eight warps per (group, head): the running maximum over the
+// chunks is a block reduction, warp w sums the chunks c = w mod 8, and warp 0
+// adds the eight partial sums in warp order, then rotates and stores.
 template <int A>
-__global__ void __launch_bounds__(128) attention_combine_hadamard_kernel(
+__global__ void __launch_bounds__(256) attention_combine_hadamard_kernel(
     QParams vp, AttnShape sh, const float* __restrict__ part, float* __restrict__ out,
     int Hq, int Hkv) {
-  const int lane = threadIdx.x & 31;
-  const int64_t w = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);  // (group, head)
-  if (w >= (int64_t)sh.groups * sh.G) return;
+  constexpr int kW = 8;
+  __shared__ float sm[kW], sl[kW];
+  __shared__ float sv[kW][32 * A];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int64_t w = blockIdx.x;  // (group, head)
   const int g = (int)(w / sh.G), h = (int)(w % sh.G);
   const int dp = vp.d_pad;
   float M = -INFINITY;
-  for (int c = 0; c < sh.n_chunks; ++c) M = fmaxf(M, partial_ptr((float*)part, dp, sh.G, sh.n_chunks, g, c, h)[0]);
+  for (int c = threadIdx.x; c < sh.n_chunks; c += 32 * kW)
+    M = fmaxf(M, partial_ptr((float*)part, dp, sh.G, sh.n_chunks, g, c, h)[0]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) sm[wib] = M;
+  __syncthreads();
+  M = sm[0];
+#pragma unroll
+  for (int i = 1; i < kW; ++i) M = fmaxf(M, sm[i]);
   float L = 0.f;
   float v[A];
 #pragma unroll
   for (int a = 0; a < A; ++a) v[a] = 0.f;
-  for (int c = 0; c < sh.n_chunks; ++c) {
+  for (int c = wib; c < sh.n_chunks; c += kW) {
     const float* pp = partial_ptr((float*)part, dp, sh.G, sh.n_chunks, g, c, h);
     if (pp[0] == -INFINITY) continue;
     const float e = expf(pp[0] - M);
     L = fmaf(e, pp[1], L);
 #pragma unroll
     for (int a = 0; a < A; ++a) v[a] = fmaf(e, pp[2 + 32 * a + lane], v[a]);
+  }
+  if (lane == 0) sl[wib] = L;
+#pragma unroll
+  for (int a = 0; a < A; ++a) sv[wib][32 * a + lane] = v[a];
+  __syncthreads();
+  if (wib != 0) return;
+  L = sl[0];
+#pragma unroll
+  for (int i = 1; i < kW; ++i) L += sl[i];
+#pragma unroll
+  for (int a = 0; a < A; ++a) {
+    float t = sv[0][32 * a + lane];
+#pragma unroll
+    for (int i = 1; i < kW; ++i) t += sv[i][32 * a + lane];
+    v[a] = t;
   }
   const float inv = L > 0.f ? 1.0f / L : 0.f;
   warp_fwht<A>(v, lane);

@@ -12,38 +12,51 @@
 
 namespace tq {
 
-// q' = Pi pad(q) and u = S q' for each query (one warp per query).
-template <int A>
-__global__ void __launch_bounds__(128) query_prep_hadamard_kernel(QParams qp,
+// q' = Pi pad(q) and u = S q' for QPB queries per block of 128 or 256
+// threads: warp w < QPB rotates query w (register FWHT), then every thread
+// forms outputs of u, each a sum over j in ascending order with coalesced
+// loads of S^T (shared by the block's queries), 32 loads in flight.
+template <int A, int QPB>
+__global__ void __launch_bounds__(256) query_prep_hadamard_kernel(QParams qp,
                                                                   const float* __restrict__ q,
                                                                   int64_t nq, int64_t ldq,
                                                                   float* __restrict__ qrot,
                                                                   float* __restrict__ u) {
-  __shared__ float qs[4][32 * A];
+  __shared__ float qs[QPB][32 * A];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int64_t w = (int64_t)blockIdx.x * 4 + wib;
-  if (w >= nq) return;
-  float v[A];
+  const int64_t q0 = (int64_t)blockIdx.x * QPB;
+  if (wib < QPB && q0 + wib < nq) {
+    const int64_t w = q0 + wib;
+    float v[A];
 #pragma unroll
-  for (int a = 0; a < A; ++a) {
-    const int j = 32 * a + lane;
-    v[a] = j < qp.d ? q[w * ldq + j] : 0.f;
-  }
-  apply_signs<A>(v, qp.dmask, lane);
-  warp_fwht<A>(v, lane);
-#pragma unroll
-  for (int a = 0; a < A; ++a) {
-    v[a] *= qp.inv_sqrt_dpad;
-    qrot[w * qp.d_pad + 32 * a + lane] = v[a];
-    qs[wib][32 * a + lane] = v[a];
-  }
-  __syncwarp();
-  if (u) {
-    for (int i = lane; i < qp.m; i += 32) {
-      float acc = 0.f;
-      for (int j = 0; j < qp.d_pad; ++j) acc = fmaf(__ldg(qp.St + (size_t)j * qp.m + i), qs[wib][j], acc);
-      u[w * qp.m + i] = acc;
+    for (int a = 0; a < A; ++a) {
+      const int j = 32 * a + lane;
+      v[a] = j < qp.d ? q[w * ldq + j] : 0.f;
     }
+    apply_signs<A>(v, qp.dmask, lane);
+    warp_fwht<A>(v, lane);
+#pragma unroll
+    for (int a = 0; a < A; ++a) {
+      v[a] *= qp.inv_sqrt_dpad;
+      qrot[w * qp.d_pad + 32 * a + lane] = v[a];
+      qs[wib][32 * a + lane] = v[a];
+    }
+  }
+  __syncthreads();
+  if (!u) return;
+  for (int i = threadIdx.x; i < qp.m; i += blockDim.x) {
+    float acc[QPB];
+#pragma unroll
+    for (int t = 0; t < QPB; ++t) acc[t] = 0.f;
+#pragma unroll 32
+    for (int j = 0; j < qp.d_pad; ++j) {
+      const float sv = __ldg(qp.St + (size_t)j * qp.m + i);
+#pragma unroll
+      for (int t = 0; t < QPB; ++t) acc[t] = fmaf(sv, qs[t][j], acc[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < QPB; ++t)
+      if (q0 + t < nq) u[(q0 + t) * qp.m + i] = acc[t];
   }
 }
 
