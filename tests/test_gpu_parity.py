@@ -41,7 +41,9 @@ def x_np(x):
     (128, "float32", tq.LAYOUT_ROW, 4096),
     (128, "bfloat16", tq.LAYOUT_BLOCK32, 1000),
     (128, "float16", tq.LAYOUT_ROW, 77),
-    (192, "float16", tq.LAYOUT_BLOCK32, 555),
+    (192, "float16", tq.LAYOUT_BLOCK32, 555),  # d_pad 256 on the tensor cores (H256 = [[H, H], [H, -H]])
+    (256, "bfloat16", tq.LAYOUT_ROW, 300),
+    (200, "float16", tq.LAYOUT_ROW, 129),      # d_pad 256 with 56 zero-filled columns
     (64, "float32", tq.LAYOUT_ROW, 300),
     (100, "float32", tq.LAYOUT_BLOCK32, 333),  # d_pad 128, 400-byte rows (thread-per-vector)
     (104, "float16", tq.LAYOUT_ROW, 129),      # d_pad 128 with 24 zero-filled columns (tensor core)

@@ -43,7 +43,9 @@ def x_np(x):
     (128, "float16", tq.LAYOUT_BLOCK32, 4096, 4, False),
     (128, "float16", tq.LAYOUT_ROW, 256, 1, False),
     (128, "float32", tq.LAYOUT_ROW, 777, 3, False),        # thread-per-vector
-    (192, "float16", tq.LAYOUT_BLOCK32, 555, 4, False),    # thread-per-vector, d_pad 256
+    (192, "float16", tq.LAYOUT_BLOCK32, 555, 4, False),    # tensor-core encoder, d_pad 256
+    (256, "bfloat16", tq.LAYOUT_ROW, 300, 2, False),       # tensor-core encoder, d_pad 256, ROW
+    (192, "float32", tq.LAYOUT_BLOCK32, 100, 3, False),    # thread-per-vector, d_pad 256
     (128, "float32", tq.LAYOUT_BLOCK32, 300, 1, False),
     (64, "float32", tq.LAYOUT_ROW, 300, 3, False),         # warp-per-vector
     (96, "float32", tq.LAYOUT_BLOCK32, 224, 2, True),      # dense rotation (BLOCK32: 32-row segments)

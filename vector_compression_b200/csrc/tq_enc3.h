@@ -64,13 +64,19 @@ inline uint32_t smem_bytes(int mode, int m) {
 
 cudaError_t launch_f16(int mode, const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,
                        cudaStream_t st);
+// Q_MSE modes at d_pad = 256 (tq_encode3_256.cuh)
+cudaError_t launch256_f16(int mode, const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,
+                          cudaStream_t st);
+cudaError_t launch256_bf16(int mode, const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,
+                           cudaStream_t st);
 cudaError_t launch_bf16(int mode, const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,
                         cudaStream_t st);
 
 // Runs the request on the tensor-core encoder if it covers it (Hadamard
-// rotation with d_pad = 128, fp16/bf16 rows 16-byte aligned, segments of a
-// multiple of 32 vectors, Q_prod with m in {64, 128} and k <= 3, Q_MSE k <= 4)
-// and returns true with the launch status in *err; returns false otherwise.
+// rotation with d_pad = 128, or Q_MSE with d_pad = 256; fp16/bf16 rows 16-byte
+// aligned, segments of a multiple of 32 vectors, Q_prod with m in {64, 128}
+// and k <= 3, Q_MSE k <= 4) and returns true with the launch status in *err;
+// returns false otherwise.
 bool try_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_vec, int64_t ld,
                 int64_t seg_len, int64_t seg_cap, int layout, uint32_t* codes, uint32_t* signs,
                 float* norms, float* rnorms, unsigned* err_word, int num_sms, cudaStream_t st,

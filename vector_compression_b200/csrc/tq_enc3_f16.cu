@@ -1,5 +1,5 @@
 // Tensor-core encode kernels for f16 input rows.
-#include "tq_encode3.cuh"
+#include "tq_encode3_256.cuh"
 
 namespace tq {
 namespace enc3 {
@@ -37,7 +37,39 @@ cudaError_t by_k(const CUtensorMap& map, const QParams& qp, const Args& a, int c
   }
 }
 
+template <int K, int MODE>
+cudaError_t launch_one256(const CUtensorMap& map, const QParams& qp, const Args& a, int ctas, cudaStream_t st) {
+  const int smem = (int)smem_bytes_256();
+  auto kern = encode_tc256_kernel<__half, K, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<ctas, kThreads, smem, st>>>(map, qp, a);
+  return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t by_k256(const CUtensorMap& map, const QParams& qp, const Args& a, int ctas, cudaStream_t st) {
+  switch (qp.k) {
+    case 1: return launch_one256<1, MODE>(map, qp, a, ctas, st);
+    case 2: return launch_one256<2, MODE>(map, qp, a, ctas, st);
+    case 3: return launch_one256<3, MODE>(map, qp, a, ctas, st);
+    case 4: return launch_one256<4, MODE>(map, qp, a, ctas, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch256_f16(int mode, const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,
+                          cudaStream_t st) {
+  switch (mode) {
+    case MODE_MSE_ROW: return by_k256<MODE_MSE_ROW>(map, qp, a, ctas, st);
+    case MODE_MSE_BLOCK: return by_k256<MODE_MSE_BLOCK>(map, qp, a, ctas, st);
+    case MODE_MSE_ROW_U: return by_k256<MODE_MSE_ROW_U>(map, qp, a, ctas, st);
+    case MODE_MSE_BLOCK_U: return by_k256<MODE_MSE_BLOCK_U>(map, qp, a, ctas, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_f16(int mode, const CUtensorMap& map, const QParams& qp, const Args& a, int ctas,
                       cudaStream_t st) {

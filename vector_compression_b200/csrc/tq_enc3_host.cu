@@ -30,7 +30,8 @@ bool try_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_v
                 int64_t seg_len, int64_t seg_cap, int layout, uint32_t* codes, uint32_t* signs,
                 float* norms, float* rnorms, unsigned* err_word, int num_sms, cudaStream_t st,
                 cudaError_t* err) {
-  if (qp.rot != TQ_ROT_HADAMARD || qp.d_pad != kDP) return false;
+  const bool dp256 = !prod && qp.d_pad == 2 * kDP;  // Q_MSE at d_pad 256 (tq_encode3_256.cuh)
+  if (qp.rot != TQ_ROT_HADAMARD || (qp.d_pad != kDP && !dp256)) return false;
   if (dt != TQ_F16 && dt != TQ_BF16) return false;
   if ((qp.d * 2) % 16 != 0 || (ld * 2) % 16 != 0 || (reinterpret_cast<uintptr_t>(x) & 15u) != 0)
     return false;
@@ -46,7 +47,7 @@ bool try_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_v
   PFN_cuTensorMapEncodeTiled enc = encode_tiled_fn();
   if (!enc) return false;
   // rows of d 16-bit values, row stride ld; boxes of 64 columns x 128 rows with
-  // the 128-byte swizzle; columns d .. 127 and rows past n_vec read as zero
+  // the 128-byte swizzle; columns d .. d_pad - 1 and rows past n_vec read as zero
   CUtensorMap map;
   const cuuint64_t dims[2] = {(cuuint64_t)qp.d, (cuuint64_t)n_vec};
   const cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
@@ -73,7 +74,10 @@ bool try_encode(const QParams& qp, bool prod, const void* x, int dt, int64_t n_v
                         : qp.unbiased ? (blk ? MODE_MSE_BLOCK_U : MODE_MSE_ROW_U)
                                       : (blk ? MODE_MSE_BLOCK : MODE_MSE_ROW);
   const int ctas = (int)std::min<int64_t>(a.n_tiles, (int64_t)num_sms);
-  *err = dt == TQ_F16 ? launch_f16(mode, map, qp, a, ctas, st) : launch_bf16(mode, map, qp, a, ctas, st);
+  if (dp256)
+    *err = dt == TQ_F16 ? launch256_f16(mode, map, qp, a, ctas, st) : launch256_bf16(mode, map, qp, a, ctas, st);
+  else
+    *err = dt == TQ_F16 ? launch_f16(mode, map, qp, a, ctas, st) : launch_bf16(mode, map, qp, a, ctas, st);
   return true;
 }
 
