@@ -238,6 +238,17 @@ def run_reference(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+def retrieval_accounting(n, d, m, nq, code_words, sign_words):
+    """Algorithmic work of the retrieval line: bytes of the Q_prod encode
+    (fp32 rows in; code and sign words, norm and residual norm out), its flop
+    (y = Pi x and z = S r: 2 d^2 + 2 m d per vector) and the scores' flop
+    (<q', C[idx]> and <S q', signs>: 2 (d + m) per (query, vector) pair)."""
+    enc_bytes = n * (d * 4 + 4 * (code_words + sign_words) + 8)
+    enc_flop = n * (2 * d * d + 2 * m * d)
+    sc_flop = nq * n * 2 * (d + m)
+    return enc_bytes, enc_flop, sc_flop
+
+
 def run_retrieval(args):
     """Retrieval set timing (one GPU): Q_prod encode of 1e6 x 1536 fp32 unit
     vectors with the dense rotation (y = Pi x and z = S r are dense
@@ -281,9 +292,7 @@ def run_retrieval(args):
     # recall@10 of the estimator's top-10 against the exact fp32 inner products
     _, _, top_i = tq.tq_scores(p, q, *out, topk=R["topk"], want_scores=False)
     recall = recall_at_k(torch, x, q, top_i, R["topk"])
-    enc_bytes = n * (d * 4 + 4 * (p.code_words + p.sign_words) + 8)
-    enc_flop = n * (2 * d * d + 2 * m * d)
-    sc_flop = nq * n * 2 * (d + m)
+    enc_bytes, enc_flop, sc_flop = retrieval_accounting(n, d, m, nq, p.code_words, p.sign_words)
     peak_tf = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] \
         if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1590.0
     line = {

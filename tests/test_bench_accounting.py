@@ -31,3 +31,12 @@ def test_storage_variants_bytes():
 def test_job_throughput_counts_every_rank():
     assert bench.job_throughput(24_431_820_800, 1, 7.5) == 24_431_820_800 / 7.5e-3 / 1e9
     assert bench.job_throughput(10 ** 9, 4, 1.0) == 4000.0
+
+
+def test_retrieval_accounting():
+    # 1e6 x 1536 unit vectors, m = 1536, b = 4 (3 MSE bits): 3 x 48 code words,
+    # 48 sign words; 1024 queries
+    enc_bytes, enc_flop, sc_flop = bench.retrieval_accounting(10**6, 1536, 1536, 1024, 3 * 48, 48)
+    assert enc_bytes == 10**6 * (1536 * 4 + 4 * 192 + 8)   # 6144 in, 776 out per vector
+    assert enc_flop == 10**6 * 2 * 1536 * 1536 * 2           # Pi x and S r
+    assert sc_flop == 1024 * 10**6 * 2 * 3072
