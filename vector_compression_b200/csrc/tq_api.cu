@@ -183,14 +183,19 @@ cudaError_t encode_dense_tc(const QParams& qp, bool prod, const void* x, int dt,
     g1.ldc = d;
     e = gemm_tc::run(g1, err, nsm, st);
     if (e != cudaSuccess) return e;
+    // Q_prod: r goes straight into a2 as the split operand of z = S r (x's
+    // split there has been consumed by the y product)
     if (layout == TQ_LAYOUT_ROW)
-      launch_quantize_rows_warp(qp, y, seg_len, seg_cap, row, rows, prod, codes, norms, rnorms, st);
+      launch_quantize_rows_warp(qp, y, seg_len, seg_cap, row, rows, prod, codes, norms, rnorms, st,
+                                prod ? a2 : nullptr);
     else
       quantize_rows_kernel<<<(unsigned)ceil_div(ceil_div(rows, 32), 4), 128, 0, st>>>(
           qp, y, seg_len, seg_cap, row, rows, layout, prod, codes, norms, rnorms);
     if (prod) {
-      e = gemm_tc::split_rows(y, d, rows, a2, st);
-      if (e != cudaSuccess) return e;
+      if (layout != TQ_LAYOUT_ROW) {  // the task-per-32-rows quantizer wrote r over y
+        e = gemm_tc::split_rows(y, d, rows, a2, st);
+        if (e != cudaSuccess) return e;
+      }
       gemm_tc::Problem g2{};
       g2.A = a2;
       g2.lda = 2 * d;

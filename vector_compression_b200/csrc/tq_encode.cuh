@@ -283,10 +283,14 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(
 // arithmetic and order as that kernel: idx = #{B_k < y}, code word p * A + a
 // = the ballot of bit p, and for Q_prod r = y - C[idx] over y with
 // rho = ||r||; the unbiased Q_MSE divides the norm by <y, C[idx]>.
+// With a2 given (Q_prod on the tensor-core dense path), r is written as the
+// [hi | lo] fp16 operand of the S r product (hi = fp16(2^8 r), lo =
+// fp16(2^8 r - hi), row stride 2 d) instead of over y.
 template <int K>
 __global__ void __launch_bounds__(256) quantize_rows_warp_kernel(
     QParams qp, float* __restrict__ y, int64_t seg_len, int64_t seg_cap, int64_t row0, int64_t nrows, bool prod,
-    uint32_t* __restrict__ codes, float* __restrict__ norms, float* __restrict__ rnorms) {
+    uint32_t* __restrict__ codes, float* __restrict__ norms, float* __restrict__ rnorms,
+    uint16_t* __restrict__ a2) {
   __shared__ SmemCodebook cb;
   load_codebook(cb, qp);
   __syncthreads();
@@ -316,7 +320,15 @@ __global__ void __launch_bounds__(256) quantize_rows_warp_kernel(
     if (prod) {
       const float r = v - c;
       rr = fmaf(r, r, rr);
-      yr[32 * a + lane] = r;
+      if (a2) {
+        const __half h = __float2half_rn(r * 256.0f);
+        const __half l = __float2half_rn(r * 256.0f - __half2float(h));
+        uint16_t* ar = a2 + w * (int64_t)(2 * d);
+        ar[32 * a + lane] = __half_as_ushort(h);
+        ar[d + 32 * a + lane] = __half_as_ushort(l);
+      } else {
+        yr[32 * a + lane] = r;
+      }
     }
   }
   if (prod) {
@@ -330,13 +342,13 @@ __global__ void __launch_bounds__(256) quantize_rows_warp_kernel(
 
 inline void launch_quantize_rows_warp(const QParams& qp, float* y, int64_t seg_len, int64_t seg_cap, int64_t row0,
                                       int64_t nrows, bool prod, uint32_t* codes, float* norms, float* rnorms,
-                                      cudaStream_t st) {
+                                      cudaStream_t st, uint16_t* a2 = nullptr) {
   const unsigned blocks = (unsigned)ceil_div(nrows, 8);
   switch (qp.k) {
 #define TQ_QRW(KK)                                                                                       \
   case KK:                                                                                              \
     quantize_rows_warp_kernel<KK><<<blocks, 256, 0, st>>>(qp, y, seg_len, seg_cap, row0, nrows, prod,  \
-                                                            codes, norms, rnorms);                      \
+                                                            codes, norms, rnorms, a2);                  \
     break;
     TQ_QRW(1)
     TQ_QRW(2)
