@@ -249,6 +249,14 @@ def retrieval_accounting(n, d, m, nq, code_words, sign_words):
     return enc_bytes, enc_flop, sc_flop
 
 
+def scores_stream_bytes(n, nq, code_words, sign_words, d):
+    """Bytes the scores stream from HBM: every block of 32 queries reads each
+    vector's code words, sign words, norm and residual norm once, plus the
+    fp32 queries and the top-10 lists out (the query operands stay in L2)."""
+    blocks = (nq + 31) // 32
+    return blocks * n * (4 * (code_words + sign_words) + 8) + nq * d * 4 + nq * 10 * 12
+
+
 def run_retrieval(args):
     """Retrieval set timing (one GPU): Q_prod encode of 1e6 x 1536 fp32 unit
     vectors with the dense rotation (y = Pi x and z = S r are dense
@@ -293,6 +301,8 @@ def run_retrieval(args):
     _, _, top_i = tq.tq_scores(p, q, *out, topk=R["topk"], want_scores=False)
     recall = recall_at_k(torch, x, q, top_i, R["topk"])
     enc_bytes, enc_flop, sc_flop = retrieval_accounting(n, d, m, nq, p.code_words, p.sign_words)
+    sc_bytes = scores_stream_bytes(n, nq, p.code_words, p.sign_words, d)
+    hbm = peaks()[0]
     peak_tf = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] \
         if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1590.0
     line = {
@@ -304,7 +314,9 @@ def run_retrieval(args):
                    "frac_of_bf16_peak": enc_flop / (enc_ms * 1e-3) / 1e12 / peak_tf},
         "scores_topk": {"ms": sc_ms, "TFLOP/s": sc_flop / (sc_ms * 1e-3) / 1e12,
                         "frac_of_bf16_peak": sc_flop / (sc_ms * 1e-3) / 1e12 / peak_tf,
-                        "pairs_per_s": nq * n / (sc_ms * 1e-3)},
+                        "pairs_per_s": nq * n / (sc_ms * 1e-3),
+                        "GB/s": sc_bytes / (sc_ms * 1e-3) / 1e9,
+                        "frac_of_hbm": sc_bytes / (sc_ms * 1e-3) / 1e9 / hbm},
         "recall_at_10": recall,
         "arithmetic": {"encode": "Pi x and S r as tcgen05 fp16 contractions of split operands (hi.lo + lo.hi + "
                                  "hi.hi and lo.S + hi.S, operands split into fp16 hi + lo), fp32 accumulation per "

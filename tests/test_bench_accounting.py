@@ -40,3 +40,10 @@ def test_retrieval_accounting():
     assert enc_bytes == 10**6 * (1536 * 4 + 4 * 192 + 8)   # 6144 in, 776 out per vector
     assert enc_flop == 10**6 * 2 * 1536 * 1536 * 2           # Pi x and S r
     assert sc_flop == 1024 * 10**6 * 2 * 3072
+
+
+def test_scores_stream_bytes():
+    # 40 queries = two 32-query blocks, each streaming the 1e6 rows of codes
+    # (48 words), signs (48 words), norm and residual norm once
+    b = bench.scores_stream_bytes(10**6, 40, 48, 48, 1536)
+    assert b == 2 * 10**6 * (4 * 96 + 8) + 40 * 1536 * 4 + 40 * 10 * 12
